@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled GEMM path on B200.
+
+One step = the whole hot path on one batch of synthetic input: pack the UE8M0 scale
+factors of A (1x128) and B (128x128) into int16 MN-major words on the GPU, then the FP8
+E4M3 block-scaled GEMM D = A * B^T at M=4096 N=7168 K=16384 (fp32 accumulate, bf16 out).
+The L2 is flushed (1 GiB write) before every timed step; the flush is outside the events.
+
+The same line also reports, each measured the same way (W warm-up, flushed L2, CUDA
+events on the launching stream): BF16 dense at the same shape, FP4 E2M1 at the same
+shape, the M-grouped FP8 MoE workload (32 experts, 32768 rows, N=4096, K=7168), the FP8
+M sweep {128, 1024, 4096} at N=K=7168, and the scale transform alone (GB/s).
+
+FLOP convention 2*M*N*K per GEMM (the pages' own timings reproduce their TFLOPS with it).
+
+--impl reference times the CPU oracle (the plain fp64 definition) on bounded row samples
+of the same FP8 workload; it is a deliberately slow reference, not a target.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import inputs  # noqa: E402
+
+METRIC = "GEMM TFLOPS (FP8 block-scaled, BF16) at 4096×7168×16384; % of B200 peak"
+M, N, K = 4096, 7168, 16384
+PAGES_FP8_TFLOPS = 861.0   # pages' FP8xFP8 figure at this shape (Ascend 950DT): context only
+PAGES_BF16_TFLOPS = 431.0
+NOMINAL_RATIO = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}  # dense tensor peak relative to bf16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["block_scaled_precision_sm_b200/csrc/gemm.cuh", "block_scaled_precision_sm_b200/csrc/ptx.cuh",
+                  "block_scaled_precision_sm_b200/csrc/api.cu"]
+
+
+def gemm_flops(m: int, n: int, k: int) -> float:
+    return 2.0 * m * n * k
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--only-headline", action="store_true", help="skip the secondary workloads")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_digest() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on these sources."""
+    p = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    s = re.search(r"sources_digest:\s*([0-9a-f]+)", txt)
+    if not t or not s or s.group(1) != sources_digest():
+        return None
+    return float(t.group(1))
+
+
+# ---------------------------------------------------------------- clocks sampler
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+                power.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- our arm
+
+class Timer:
+    """Per-step CUDA events on the launching stream, L2 flushed before each step."""
+
+    def __init__(self, torch, flush_bytes=1 << 30):
+        self.torch = torch
+        self.flush = torch.empty(flush_bytes, dtype=torch.uint8, device="cuda")
+
+    def run(self, fn, warmup: int, steps: int, marks: int = 1):
+        torch = self.torch
+        for _ in range(warmup):
+            self.flush.zero_()
+            fn(None)
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(marks + 1)] for _ in range(steps)]
+        for i in range(steps):
+            self.flush.zero_()
+            fn(evs[i])
+        torch.cuda.synchronize()
+        spans = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(marks)] for i in range(steps)])
+        return spans  # ms, [steps, marks]
+
+
+def fp8_device_problem(torch, m, n, k, seed):
+    p = inputs.dense_fp8_problem(m, n, k, seed=seed)
+    dev = {key: torch.from_numpy(p[key]).cuda() for key in ("A", "sfa", "B", "sfb")}
+    return p, dev
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_scaled_precision_sm_b200 import ops
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks, peak_kind = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    timer = Timer(torch)
+    kb = K // 128
+    # independent problem per rank (weak scaling): the seed differs by rank
+    p, dev = fp8_device_problem(torch, M, N, K, seed=100 + 7 * rank)
+    sfa_w = torch.empty(((kb + 1) // 2, ops.sf_ld(M)), dtype=torch.int16, device="cuda")
+    sfb_w = torch.empty(((kb + 1) // 2, ops.sf_ld(N // 128)), dtype=torch.int16, device="cuda")
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+
+    def step(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.transform_sf_ue8m0(dev["sfa"], out=sfa_w)
+        ops.transform_sf_ue8m0(dev["sfb"], out=sfb_w)
+        if ev is not None:
+            ev[1].record()
+        ops.gemm_fp8_nt(dev["A"], sfa_w, dev["B"], sfb_w, D, sfb_gran_n=128)
+        if ev is not None:
+            ev[2].record()
+
+    # warm-up + timed region bracketed by barrier and synchronize on both sides
+    for _ in range(args.warmup):
+        timer.flush.zero_()
+        step(None)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    launches0 = ops.kernel_launches()
+    wall0 = time.perf_counter()
+    spans = timer.run(step, 0, args.steps, marks=2)
+    wall = time.perf_counter() - wall0
+    launches = ops.kernel_launches() - launches0
+    clocks = sampler.stop()
+    torch.cuda.synchronize()
+    barrier()
+    status = ops.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    step_ms = max_over_ranks(float(spans.sum(axis=1).mean()))
+    gemm_ms = max_over_ranks(float(spans[:, 1].mean()))
+    flops = gemm_flops(M, N, K)
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    fp8_peak = peaks["bf16_tflops"] * NOMINAL_RATIO["fp8"]
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    traffic = profiled_traffic("gemm_fp8_4096x7168x16384.md")
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": round(value / world / PAGES_FP8_TFLOPS, 3),
+        "vs_baseline_note": "per-GPU value / the pages' 861 TFLOPS FP8xFP8 at this shape on an Ascend 950DT "
+                            "(another machine: context, not the target)",
+        "dtype": "e4m3 x ue8m0 scales, fp32 accumulate, bf16 out", "data": "synthetic",
+        "config": {"workload": "fp8_block_scaled_gemm_nt 4096x7168x16384 (sf transform + gemm)", "M": M, "N": N,
+                   "K": K, "sfa": "1x128 ue8m0", "sfb": "128x128 ue8m0",
+                   "l2": "flushed by a 1 GiB write before every step, outside the events",
+                   "parallelism": f"one independent problem per GPU x{world}"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
+                     "frac_of_sustained": round(achieved / (peaks.get("bf16_tflops_sustained", 1400.0) * 2), 4),
+                     "kernel": "gemm_kernel<FP8,224>", "kernel_ms": round(gemm_ms, 5)},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 3),
+    }
+
+    # end to end through the public API: pinned host inputs -> GPU -> host result, every step
+    pin = {key: torch.from_numpy(p[key]).pin_memory() for key in ("A", "sfa", "B", "sfb")}
+    D_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = D_host.numel() * D_host.element_size()
+
+    def e2e_step(ev):
+        if ev is not None:
+            ev[0].record()
+        for key in pin:
+            dev[key].copy_(pin[key], non_blocking=True)
+        ops.gemm_fp8_nt(dev["A"], dev["sfa"], dev["B"], dev["sfb"], D, sfb_gran_n=128)
+        D_host.copy_(D, non_blocking=True)
+        if ev is not None:
+            ev[1].record()
+
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = max_over_ranks(float(timer.run(e2e_step, 2, e2e_steps)[:, 0].mean()))
+    line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                   "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                   "api": "ops.gemm_fp8_nt with uint8 UE8M0 scales (packed inside the call)"}
+
+    if world == 1 and not args.only_headline:
+        line["secondary"] = secondary(torch, ops, timer, args, peaks, peak_kind)
+        line["cpu_baseline"] = cpu_baseline(p)
+    if ops.device_status() != 0:
+        raise RuntimeError("device status after secondary workloads")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _gemm_entry(name, flops, ms, peak, extra=None):
+    d = {"tflops": round(flops / (ms * 1e-3) / 1e12, 1), "ms": round(ms, 5), "peak_tflops": round(peak, 1),
+         "frac": round(flops / (ms * 1e-3) / 1e12 / peak, 4)}
+    if extra:
+        d.update(extra)
+    return name, d
+
+
+def secondary(torch, ops, timer, args, peaks, peak_kind):
+    reps = max(5, min(args.steps, 30))
+    out = {"peak_source": f"{peak_kind} bf16 burst x nominal dtype ratio"}
+    bf16_peak = peaks["bf16_tflops"]
+
+    # BF16 dense, same shape
+    p = inputs.dense_bf16_problem(M, N, K, seed=2)
+    A = torch.from_numpy(p["A"]).cuda().view(torch.bfloat16)
+    B = torch.from_numpy(p["B"]).cuda().view(torch.bfloat16)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    del p
+
+    def f_bf16(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.gemm_bf16_nt(A, B, D)
+        if ev is not None:
+            ev[1].record()
+
+    ms = float(timer.run(f_bf16, args.warmup, reps)[:, 0].mean())
+    k, v = _gemm_entry("bf16_4096x7168x16384", gemm_flops(M, N, K), ms, bf16_peak,
+                       {"vs_pages_431": round(gemm_flops(M, N, K) / (ms * 1e-3) / 1e12 / PAGES_BF16_TFLOPS, 3),
+                        "traffic": profiled_traffic("gemm_bf16_4096x7168x16384.md")})
+    out[k] = v
+    del A, B
+
+    # FP4, same shape
+    p = inputs.dense_fp4_problem(M, N, K, seed=6)
+    d4 = {key: torch.from_numpy(p[key]).cuda() for key in ("A", "sfa", "B", "sfb")}
+    sa = ops.transform_sf_ue8m0(d4["sfa"])
+    sb = ops.transform_sf_ue8m0(d4["sfb"])
+    del p
+
+    def f_fp4(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.gemm_fp4_nt(d4["A"], sa, d4["B"], sb, D)
+        if ev is not None:
+            ev[1].record()
+
+    ms = float(timer.run(f_fp4, args.warmup, reps)[:, 0].mean())
+    k, v = _gemm_entry("fp4_4096x7168x16384", gemm_flops(M, N, K), ms, bf16_peak * NOMINAL_RATIO["fp4"])
+    out[k] = v
+    del d4, sa, sb
+
+    # FP8 M sweep at N = K = 7168
+    sweep = {}
+    for m in (128, 1024, 4096):
+        p, dv = fp8_device_problem(torch, m, 7168, 7168, seed=30 + m)
+        sa = ops.transform_sf_ue8m0(dv["sfa"])
+        sb = ops.transform_sf_ue8m0(dv["sfb"])
+        Dm = torch.empty((m, 7168), dtype=torch.bfloat16, device="cuda")
+
+        def f_sw(ev, dv=dv, sa=sa, sb=sb, Dm=Dm):
+            if ev is not None:
+                ev[0].record()
+            ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, Dm)
+            if ev is not None:
+                ev[1].record()
+
+        ms = float(timer.run(f_sw, args.warmup, reps)[:, 0].mean())
+        bytes_min = m * 7168 + 7168 * 7168 + 2 * m * 7168
+        fl = gemm_flops(m, 7168, 7168)
+        sweep[str(m)] = {"tflops": round(fl / (ms * 1e-3) / 1e12, 1), "ms": round(ms, 5),
+                         "frac_tensor": round(fl / (ms * 1e-3) / 1e12 / (bf16_peak * 2), 4),
+                         "hbm_gbs_min_bytes": round(bytes_min / (ms * 1e-3) / 1e9, 1)}
+        del p, dv, sa, sb, Dm
+    out["fp8_m_sweep_n7168_k7168"] = sweep
+
+    # M-grouped FP8 MoE workload
+    g = inputs.grouped_fp8_problem(32, 32768, 4096, 7168, seed=8)
+    dg = {key: torch.from_numpy(g[key]).cuda() for key in ("A", "sfa", "B", "m_indices")}
+    sfa_g = ops.transform_sf_ue8m0(dg["sfa"])
+    sfb_g = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(g["sfb"][e]).cuda()) for e in range(32)])
+    Dg = torch.empty((g["M"], 4096), dtype=torch.bfloat16, device="cuda")
+
+    def f_grp(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.m_grouped_gemm_fp8_nt_contiguous(dg["A"], sfa_g, dg["B"], sfb_g, dg["m_indices"], Dg)
+        if ev is not None:
+            ev[1].record()
+
+    ms = float(timer.run(f_grp, args.warmup, reps)[:, 0].mean())
+    fl_valid = gemm_flops(32768, 4096, 7168)
+    fl_padded = gemm_flops(g["M"], 4096, 7168)
+    k, v = _gemm_entry("grouped_fp8_32x32768x4096x7168", fl_valid, ms, bf16_peak * 2,
+                       {"m_total_padded": int(g["M"]),
+                        "tflops_incl_padding": round(fl_padded / (ms * 1e-3) / 1e12, 1)})
+    out[k] = v
+
+    # scale transform alone: config-3 SFA (fp32 scales [M_total, 56]) -> int16 words
+    s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()
+    w = torch.empty((28, ops.sf_ld(g["M"])), dtype=torch.int16, device="cuda")
+    del g, dg, Dg
+
+    def f_sf(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.transform_sf_ue8m0(s32, out=w)
+        if ev is not None:
+            ev[1].record()
+
+    ms = float(timer.run(f_sf, args.warmup, reps)[:, 0].mean())
+    moved = s32.numel() * 4 + w.numel() * 2
+    out["sf_transform_fp32_36864x56"] = {"gbs": round(moved / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 5),
+                                         "bytes": int(moved), "hbm_peak_gbs": peaks["hbm_gbs"],
+                                         "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    return out
+
+
+def cpu_baseline(p, budget_s: float = 10.0):
+    """The oracle as it stands, on leading rows of the same FP8 problem, for about budget_s."""
+    import oracle
+
+    oracle.build()
+    rows_done, t_total = 0, 0.0
+    chunk = 16
+    while t_total < budget_s and rows_done < M:
+        r = np.arange(rows_done, min(rows_done + chunk, M), dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"], gran_n=128, rows=r)
+        t_total += time.perf_counter() - t0
+        rows_done += len(r)
+    return {"value": round(gemm_flops(rows_done, N, K) / t_total / 1e12, 6), "unit": "TFLOPS",
+            "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"first {rows_done} of {M} rows x all {N} columns of the FP8 {M}x{N}x{K} GEMM "
+                      f"({t_total:.1f} s)"}
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    p = inputs.dense_fp8_problem(M, N, K, seed=100)
+    rows_per_step = 2
+
+    def step(i):
+        r0 = (i * rows_per_step) % M
+        oracle.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"], gran_n=128,
+                        rows=np.arange(r0, r0 + rows_per_step, dtype=np.int32))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = gemm_flops(rows_per_step, N, K) / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic",
+            "config": {"workload": "fp8_block_scaled_gemm_nt 4096x7168x16384", "M": M, "N": N, "K": K,
+                       "sample_per_step": f"{rows_per_step} rows x {N} columns"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": oracle.threads(),
+                             "kind": "oracle", "sample": f"{rows_per_step} rows x {N} columns per step"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

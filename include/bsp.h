@@ -1,0 +1,158 @@
+/*
+ * bsp.h — C ABI of libbsp.so: block-scaled GEMM D = A * B^T on one B200 (sm_100a).
+ *
+ * Operations (the DeepGEMM-style calls the pages list):
+ *   - dense GEMM in BF16, FP8 and FP4, and an M-grouped GEMM for mixture-of-experts
+ *     layers ("DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section
+ *     "Cobertura de operações e a lacuna declarada no repositório"; "DeepSeek lanza
+ *     kernels de DeepGEMM para Huawei Ascend 950", section "Qué incluye el lanzamiento");
+ *   - the UE8M0 scale-factor layout transform: each pair of UE8M0 factors along K in
+ *     one 16-bit integer, stored MN-major ("DeepSeek lanza kernels de DeepGEMM para
+ *     Huawei Ascend 950", section "Qué incluye el lanzamiento"; "DeepGEMM-Ascend cobre
+ *     quantas operações no Ascend 950?", section "Fatores de escala FP8 e o formato
+ *     UE8M0 no Ascend").
+ *
+ * Conventions shared by every call
+ *   - "NT": A is M x K row-major (K contiguous), B is N x K row-major, D is M x N
+ *     row-major bf16.  Leading dimensions (lda, ldb, ldd, ld_sf*) are in ELEMENTS of
+ *     the stored type (bytes for FP8 and for packed FP4, 2-byte units for bf16/int16).
+ *   - Every pointer is a DEVICE pointer owned by the caller; the library never frees
+ *     or retains caller memory.  Work is enqueued asynchronously on `stream` (a
+ *     cudaStream_t passed as void*; NULL = legacy default stream) on the current device.
+ *   - Argument errors are returned synchronously and nothing is launched.  Launch
+ *     failures return BSP_ERR_CUDA.  Faults found while the kernels run (a wait that
+ *     timed out, a malformed scale or expert index) are latched in a per-device status
+ *     word and reported by bsp_get_device_status().
+ *   - Alignment: base pointers 16-byte aligned; lda/ldb/ldd/ld_sf* times the element
+ *     size a multiple of 16 bytes (the tensor-memory-accelerator copy rule).
+ *   - M and N may take any positive value (rows and columns past them are neither
+ *     read as data nor written); K has the per-call rule stated below.
+ *
+ * Packed scale-factor layout ("SF words"): for a matrix with MN scale rows and KB scale
+ * blocks along K, the SF tensor is int16 [ceil(KB/2)][ld], with
+ *     word(j, r) = sf[j*ld + r] = e[r][2j] | e[r][2j+1] << 8
+ * where e are biased UE8M0 bytes (scale = 2^(e-127)), the lower K block in the low
+ * byte (a reading: the pages give no byte order).  ld >= MN; entries r >= MN and the
+ * high byte of the last word when KB is odd are 0.
+ */
+#ifndef BSP_H
+#define BSP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BSP_OK = 0,
+    BSP_ERR_ARG = -1,          /* null pointer, negative size, bad enum value */
+    BSP_ERR_ALIGN = -2,        /* pointer or leading dimension breaks the 16-byte rule */
+    BSP_ERR_SHAPE = -3,        /* K (or M_total) breaks its multiple-of rule, ld too small */
+    BSP_ERR_UNSUPPORTED = -4,  /* no B200 (sm_100) device current, or size out of range */
+    BSP_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed */
+    BSP_ERR_TIMEOUT = -6,      /* device: a pipeline wait gave up (latched) */
+    BSP_ERR_DEVICE_CHECK = -7  /* device: bad scale value or expert index seen (latched) */
+} bsp_status;
+
+/*
+ * gemm_bf16_nt — D[m,n] = bf16( sum_k A[m,k] * B[n,k] ), fp32 accumulation.
+ *   A  bf16 [M][lda], B bf16 [N][ldb], D bf16 [M][ldd].
+ *   K: any positive multiple of 8 (so that rows stay 16-byte aligned).
+ */
+int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K,
+                 int64_t lda, int64_t ldb, int64_t ldd, void* stream);
+
+/*
+ * gemm_fp8_nt — FP8 E4M3 GEMM with fine-grained UE8M0 scales along K
+ * ("DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Fatores de
+ * escala FP8 e o formato UE8M0 no Ascend"):
+ *   D[m,n] = bf16( sum_kb 2^(ea[m,kb]-127) * 2^(eb[n/g,kb]-127)
+ *                  * sum_{k in block kb} A[m,k] * B[n,k] ),  blocks of 128 along K.
+ *   A   E4M3 bytes [M][lda];  B  E4M3 bytes [N][ldb];  D bf16 [M][ldd].
+ *   sfa SF words for MN = M rows, KB = K/128:            int16 [ceil(KB/2)][ld_sfa].
+ *   sfb SF words for MN = ceil(N/g) rows, g = sfb_gran_n: int16 [ceil(KB/2)][ld_sfb].
+ *       sfb_gran_n = 128: one scale per 128x128 block of B (weights);
+ *       sfb_gran_n = 1:   one scale per row of B and 128 K.
+ *   K: positive multiple of 128.  fp32 accumulation; one accumulation order.
+ */
+int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D,
+                int M, int N, int K, int64_t lda, int64_t ldb, int64_t ldd,
+                int64_t ld_sfa, int64_t ld_sfb, int sfb_gran_n, void* stream);
+
+/*
+ * gemm_fp4_nt — FP4 E2M1 GEMM, one UE8M0 scale per 32 K elements for every row of A
+ * and of B (pages: FP4 coverage, section "Cobertura de operações ..." of "DeepGEMM-Ascend
+ * cobre quantas operações no Ascend 950?"):
+ *   D[m,n] = bf16( sum_kb 2^(ea[m,kb]-127) * 2^(eb[n,kb]-127) * sum_{k in kb} A[m,k]*B[n,k] ).
+ *   A, B: two E2M1 values per byte, even K index in the low nibble: [M][lda], [N][ldb]
+ *         with lda, ldb in BYTES (>= K/2).
+ *   sfa SF words for MN = M, KB = K/32; sfb SF words for MN = N, KB = K/32.
+ *   K: positive multiple of 64.
+ */
+int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D,
+                int M, int N, int K, int64_t lda, int64_t ldb, int64_t ldd,
+                int64_t ld_sfa, int64_t ld_sfb, void* stream);
+
+/*
+ * m_grouped_gemm_fp8_nt_contiguous — M-grouped FP8 GEMM for mixture-of-experts layers
+ * ("DeepSeek lanza kernels de DeepGEMM para Huawei Ascend 950", section "Qué incluye el
+ * lanzamiento": grouped operations for mixture-of-experts models).  The rows of all
+ * experts are concatenated along M; row m uses expert g = m_indices[m]:
+ *   D[m,n] = FP8 formula above with B := B[g], SFB := SFB[g]   if g >= 0,
+ *   D[m,n] = 0                                                  if g == -1 (padding).
+ *   A [M_total][K] E4M3 (row stride K); sfa SF words for MN = M_total, ld_sfa.
+ *   B [G][N][K] E4M3 (contiguous); sfb [G][ceil(KB/2)][ld_sfb] SF words per expert with
+ *     MN = ceil(N/sfb_gran_n); D [M_total][N] bf16 (row stride N).
+ *   m_indices int32 [M_total]: every 128-row block [128i, 128i+128) holds one expert's
+ *     rows followed by -1 padding rows only; its first row is not padding.
+ *   M_total: positive multiple of 128.  K: positive multiple of 128.  1 <= G.
+ *   A block that breaks the layout rule (index >= G, < -1, or a second expert in the
+ *   block) latches BSP_ERR_DEVICE_CHECK; its rows hold unspecified values.
+ */
+int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void* B, const void* sfb,
+                                     void* D, const int32_t* m_indices, int M_total, int N, int K,
+                                     int G, int64_t ld_sfa, int64_t ld_sfb, int sfb_gran_n,
+                                     void* stream);
+
+/*
+ * transform_sf_ue8m0 — scale factors [mn][kb] (row stride ld_in) into SF words
+ * int16 [ceil(kb/2)][ld_out] (layout above).
+ *   in_kind 0: fp32 scales, each an exact positive normal power of two; its biased
+ *              exponent (bits 30..23) is the UE8M0 byte.  A value that is not such a
+ *              power of two latches BSP_ERR_DEVICE_CHECK (its byte is still written).
+ *   in_kind 1: uint8 biased UE8M0 bytes, copied as they are.
+ *   ld_out >= mn and ld_out*2 a multiple of 16 bytes; sf_out must not overlap sf_in.
+ * The caller decides whether a tensor is already packed ("reuse or convert",
+ * "Fatores de escala FP8 e o formato UE8M0 no Ascend"); this call always converts.
+ */
+int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in,
+                       void* sf_out, int64_t ld_out, void* stream);
+
+/*
+ * bsp_get_device_status — synchronises `stream`, then returns and clears the status
+ * word latched by kernels on the current device (BSP_OK if nothing was latched).
+ */
+int bsp_get_device_status(void* stream);
+
+/* bsp_status_string — static description of a status code (never NULL). */
+const char* bsp_status_string(int status);
+
+/*
+ * bsp_set_wait_timeout_ns — upper bound for every device-side pipeline wait (default
+ * 2e9 ns).  A wait that exceeds it latches BSP_ERR_TIMEOUT and the kernel winds down.
+ * Returns the previous value.
+ */
+uint64_t bsp_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * bsp_kernel_launches — number of kernels this library has launched in this process
+ * (all devices, all calls).  For the bench's launch count.
+ */
+uint64_t bsp_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSP_H */

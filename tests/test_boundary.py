@@ -1,0 +1,88 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every symbol bsp.h
+declares, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bsp.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|uint64_t|char\s*\*|const char\s*\*)\s*\**\s*(\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_scaled_precision_sm_b200 import _lib, build
+
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for n in ("gemm_bf16_nt", "gemm_fp8_nt", "gemm_fp4_nt", "m_grouped_gemm_fp8_nt_contiguous",
+              "transform_sf_ue8m0", "bsp_get_device_status", "bsp_status_string"):
+        assert n in names
+
+
+def test_exports_every_declared_symbol(lib):
+    from block_scaled_precision_sm_b200 import _lib
+
+    for n in _declared():
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings(lib):
+    from block_scaled_precision_sm_b200 import _lib
+
+    for code in range(-7, 1):
+        assert _lib.describe(code)
+    assert _lib.describe(123) == "unknown status"
+
+
+def test_rejects_bad_arguments_without_gpu(lib):
+    vp = ctypes.c_void_p
+    good = vp(0x10000)  # never dereferenced: validation fails first
+    odd = vp(0x10001)
+    # null pointer, empty sizes
+    assert lib.gemm_fp8_nt(None, good, good, good, good, 128, 128, 128, 128, 128, 128, 128, 8, 128, None) == -1
+    assert lib.gemm_fp8_nt(good, good, good, good, good, 0, 128, 128, 128, 128, 128, 128, 8, 128, None) == -1
+    assert lib.gemm_bf16_nt(good, good, good, 128, -1, 64, 64, 64, 64, None) == -1
+    # K breaks its rule
+    assert lib.gemm_fp8_nt(good, good, good, good, good, 128, 128, 100, 128, 128, 128, 128, 8, 128, None) == -3
+    assert lib.gemm_fp4_nt(good, good, good, good, good, 128, 128, 96, 48, 48, 128, 128, 128, None) == -3
+    assert lib.gemm_bf16_nt(good, good, good, 128, 128, 12, 16, 16, 128, None) == -3
+    # misaligned pointer / leading dimension
+    assert lib.gemm_fp8_nt(odd, good, good, good, good, 128, 128, 128, 128, 128, 128, 128, 8, 128, None) == -2
+    assert lib.gemm_bf16_nt(good, good, good, 128, 128, 64, 68, 64, 128, None) == -2
+    # ld too small
+    assert lib.gemm_fp8_nt(good, good, good, good, good, 128, 128, 256, 128, 256, 128, 128, 8, 128, None) == -3
+    # bad granularity
+    assert lib.gemm_fp8_nt(good, good, good, good, good, 128, 128, 128, 128, 128, 128, 128, 8, 64, None) == -1
+    # grouped: M_total not a multiple of 128, G < 1
+    assert lib.m_grouped_gemm_fp8_nt_contiguous(good, good, good, good, good, good, 100, 128, 128, 2, 128, 8, 128,
+                                                None) == -3
+    assert lib.m_grouped_gemm_fp8_nt_contiguous(good, good, good, good, good, good, 128, 128, 128, 0, 128, 8, 128,
+                                                None) == -1
+    # transform: kind, ld_out, overlap
+    assert lib.transform_sf_ue8m0(good, 2, 8, 8, 8, vp(0x20000), 8, None) == -1
+    assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 4, None) == -3
+    assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 12, None) == -2
+    assert lib.transform_sf_ue8m0(good, 1, 64, 8, 8, vp(0x10010), 64, None) == -1
+
+
+def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
+    from block_scaled_precision_sm_b200 import _lib
+
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load()

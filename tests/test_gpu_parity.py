@@ -1,0 +1,249 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Inputs come from the seeded generators in ``inputs``; the GPU path packs the scale
+factors with its own transform kernel, the oracle reads the unpacked UE8M0 bytes.
+Bit-exact where the result is unique (scale transform, identity closed form, G=1
+grouped = dense); the stated GEMM tolerance (tests/parity.py) elsewhere.
+"""
+
+import numpy as np
+import pytest
+
+import inputs
+
+from parity import bf16_to_f64, check_gemm, to_dev
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def ops():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_scaled_precision_sm_b200.ops as ops
+
+    assert ops.device_status() == 0
+    return ops
+
+
+def _status_ok(ops):
+    st = ops.device_status()
+    assert st == 0, f"device status {st}"
+
+
+
+# ------------------------------------------------------------------ SF transform
+
+@pytest.mark.parametrize("mn,kb,ld_pad", [(256, 8, 0), (37, 5, 3), (1, 1, 7), (4096, 128, 0), (300, 130, 12)])
+def test_transform_bit_exact_u8(ops, orc, mn, kb, ld_pad):
+    rng = np.random.default_rng(mn + kb)
+    e = rng.integers(0, 255, size=(mn, kb), dtype=np.uint8)
+    ld = (mn + 7) // 8 * 8 + 8 * ld_pad
+    got = ops.transform_sf_ue8m0(to_dev(e), ld_out=ld)
+    _status_ok(ops)
+    assert np.array_equal(got.cpu().numpy(), orc.sf_pack(e, ld_out=ld))
+
+
+@pytest.mark.parametrize("mn,kb", [(36864, 56), (7168, 512), (129, 3)])
+def test_transform_bit_exact_fp32(ops, orc, mn, kb):
+    rng = np.random.default_rng(kb)
+    e = rng.integers(1, 255, size=(mn, kb), dtype=np.uint8)
+    s = np.ldexp(np.float32(1.0), e.astype(np.int32) - 127).astype(np.float32)
+    got = ops.transform_sf_ue8m0(to_dev(s))
+    _status_ok(ops)
+    ld = (mn + 7) // 8 * 8
+    assert np.array_equal(got.cpu().numpy(), orc.sf_pack(orc.fp32_scales_to_ue8m0(s), ld_out=ld))
+
+
+def test_transform_flags_bad_scale(ops):
+    s = np.ones((16, 4), np.float32)
+    s[3, 2] = 3.0
+    ops.transform_sf_ue8m0(to_dev(s))
+    assert ops.device_status() == -7
+    _status_ok(ops)  # cleared
+
+
+def test_reuse_or_convert(ops):
+    e = to_dev(np.full((256, 8), 127, np.uint8))
+    packed = ops.packed_sf(e, 256, 8)
+    assert packed.dtype == torch.int16 and tuple(packed.shape) == (4, 256)
+    assert ops.packed_sf(packed, 256, 8) is packed  # already packed: reused, not converted
+
+
+# ------------------------------------------------------------------ FP8
+
+def _fp8_case(ops, orc, m, n, k, seed, gran, fp32_scales=False):
+    p = inputs.dense_fp8_problem(m, n, k, seed=seed, b_block_rows=gran)
+    sfa, sfb = p["sfa"], p["sfb"]
+    if fp32_scales:
+        sfa = np.ldexp(np.float32(1), sfa.astype(np.int32) - 127).astype(np.float32)
+        sfb = np.ldexp(np.float32(1), sfb.astype(np.int32) - 127).astype(np.float32)
+    ldd = (n + 7) // 8 * 8  # rows of D must start 16-byte aligned
+    D = torch.empty((m, ldd), dtype=torch.bfloat16, device="cuda")[:, :n]
+    ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(sfa), to_dev(p["B"]), to_dev(sfb), D, sfb_gran_n=gran)
+    _status_ok(ops)
+    ref = orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"], gran_n=gran)
+    return check_gemm(bf16_to_f64(D), ref, f"fp8 {m}x{n}x{k} gran {gran}")
+
+
+def test_fp8_config0(ops, orc):
+    # 256 x 512 x 1024, 1x128 A scales, 128x128 B scales, scales packed on the GPU
+    _fp8_case(ops, orc, 256, 512, 1024, seed=0, gran=128)
+
+
+@pytest.mark.parametrize("m,n,k,gran", [(200, 300, 384, 128), (130, 232, 256, 1), (1, 1024, 128, 128),
+                                        (300, 8, 256, 1), (129, 449, 640, 1), (384, 672, 2048, 128)])
+def test_fp8_ragged(ops, orc, m, n, k, gran):
+    _fp8_case(ops, orc, m, n, k, seed=m + n, gran=gran)
+
+
+def test_fp8_fp32_scale_inputs(ops, orc):
+    _fp8_case(ops, orc, 256, 448, 512, seed=3, gran=128, fp32_scales=True)
+
+
+def test_fp8_identity_bit_exact(ops, orc):
+    # A = I (E4M3 1.0 = 0x38) with unit scales: D = B^T * scale exactly, representable in bf16
+    k = 256
+    A = np.zeros((k, k), np.uint8)
+    A[np.arange(k), np.arange(k)] = 0x38
+    sfa = np.full((k, 2), 127, np.uint8)
+    rng = np.random.default_rng(9)
+    n = 448
+    B = rng.integers(0, 256, size=(n, k), dtype=np.uint8)
+    B = np.where((B & 0x7F) == 0x7F, B & 0xFE, B).astype(np.uint8)
+    sfb = rng.integers(118, 136, size=(4, 2), dtype=np.uint8)
+    D = ops.gemm_fp8_nt(to_dev(A), to_dev(sfa), to_dev(B), to_dev(sfb), sfb_gran_n=128)
+    _status_ok(ops)
+    ref = orc.gemm_fp8(A, sfa, B, sfb, gran_n=128)
+    assert np.array_equal(D.view(torch.int16).cpu().numpy().view(np.uint16), orc.bf16_round(ref))
+
+
+@pytest.mark.parametrize("m,n,gran", [(1, 8, 128), (1, 1, 1), (3, 17, 128)])
+def test_fp8_degenerate_shapes_bit_exact(ops, orc, m, n, gran):
+    # a handful of outputs: each row of A picks one K column (E4M3 1.0), so every output is
+    # one decoded B value times its scales, exactly representable in bf16
+    k = 256
+    rng = np.random.default_rng(m * 31 + n)
+    A = np.zeros((m, k), np.uint8)
+    A[np.arange(m), rng.integers(0, k, m)] = 0x38
+    B = rng.integers(0, 256, size=(n, k), dtype=np.uint8)
+    B = np.where((B & 0x7F) == 0x7F, B & 0xFE, B).astype(np.uint8)
+    sfa = rng.integers(120, 134, size=(m, 2), dtype=np.uint8)
+    sfb = rng.integers(120, 134, size=(-(-n // gran), 2), dtype=np.uint8)
+    ldd = (n + 7) // 8 * 8
+    D = torch.zeros((m, ldd), dtype=torch.bfloat16, device="cuda")
+    ops.gemm_fp8_nt(to_dev(A), to_dev(sfa), to_dev(B), to_dev(sfb), D[:, :n], sfb_gran_n=gran)
+    _status_ok(ops)
+    got = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got[:, :n], orc.bf16_round(orc.gemm_fp8(A, sfa, B, sfb, gran_n=gran)))
+    assert not got[:, n:].any()  # nothing written past column N
+
+
+def test_fp8_single_scale_localises(ops, orc):
+    # unit scales everywhere but one (row, K-block) of A and one (N-block, K-block) of B
+    p = inputs.dense_fp8_problem(256, 448, 512, seed=12)
+    sfa = np.full_like(p["sfa"], 127)
+    sfb = np.full_like(p["sfb"], 127)
+    sfa[77, 3] = 131
+    sfb[2, 1] = 124
+    D = ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(sfa), to_dev(p["B"]), to_dev(sfb), sfb_gran_n=128)
+    _status_ok(ops)
+    check_gemm(bf16_to_f64(D), orc.gemm_fp8(p["A"], sfa, p["B"], sfb), "single-scale")
+
+
+# ------------------------------------------------------------------ BF16 / FP4
+
+@pytest.mark.parametrize("m,n,k", [(256, 448, 512), (130, 200, 200), (128, 224, 64), (300, 1000, 1000)])
+def test_bf16(ops, orc, m, n, k):
+    p = inputs.dense_bf16_problem(m, n, k, seed=m)
+    A = to_dev(p["A"], torch.bfloat16)
+    B = to_dev(p["B"], torch.bfloat16)
+    ldd = (n + 7) // 8 * 8
+    D = torch.empty((m, ldd), dtype=torch.bfloat16, device="cuda")[:, :n]
+    ops.gemm_bf16_nt(A, B, D)
+    _status_ok(ops)
+    check_gemm(bf16_to_f64(D), orc.gemm_bf16(p["A"], p["B"]), f"bf16 {m}x{n}x{k}")
+
+
+def test_bf16_identity_bit_exact(ops, orc):
+    k = 128
+    eye = np.zeros((k, k), np.float32)
+    eye[np.arange(k), np.arange(k)] = 1.0
+    A = inputs.bf16_operand(eye)
+    B = inputs.bf16_operand(np.random.default_rng(1).standard_normal((224, k)).astype(np.float32))
+    D = ops.gemm_bf16_nt(to_dev(A, torch.bfloat16), to_dev(B, torch.bfloat16))
+    _status_ok(ops)
+    assert np.array_equal(D.view(torch.int16).cpu().numpy().view(np.uint16), B.T)
+
+
+@pytest.mark.parametrize("m,n,k", [(256, 448, 1024), (130, 250, 320), (128, 224, 64), (256, 512, 4096)])
+def test_fp4(ops, orc, m, n, k):
+    p = inputs.dense_fp4_problem(m, n, k, seed=n)
+    ldd = (n + 7) // 8 * 8
+    D = torch.empty((m, ldd), dtype=torch.bfloat16, device="cuda")[:, :n]
+    ops.gemm_fp4_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]), D)
+    _status_ok(ops)
+    check_gemm(bf16_to_f64(D), orc.gemm_fp4(p["A"], p["sfa"], p["B"], p["sfb"]), f"fp4 {m}x{n}x{k}")
+
+
+# ------------------------------------------------------------------ grouped
+
+def _grouped(ops, p):
+    return ops.m_grouped_gemm_fp8_nt_contiguous(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]),
+                                                to_dev(p["sfb"]), to_dev(p["m_indices"]))
+
+
+@pytest.mark.parametrize("counts,n,k", [([100, 0, 150, 50], 448, 512), ([128, 256, 1, 127, 300], 256, 384)])
+def test_grouped(ops, orc, counts, n, k):
+    p = inputs.grouped_fp8_problem(len(counts), sum(counts), n, k, seed=len(counts), counts=counts)
+    D = _grouped(ops, p)
+    _status_ok(ops)
+    got = bf16_to_f64(D)
+    ref = orc.gemm_grouped_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["m_indices"])
+    check_gemm(got, ref, "grouped")
+    pad = p["m_indices"] < 0
+    assert np.all(got[pad] == 0.0)  # padding rows are exactly zero
+
+
+def test_grouped_padding_rows_zero_whatever_a_holds(ops, orc):
+    p = inputs.grouped_fp8_problem(2, 200, 224, 256, seed=5, counts=[70, 130])
+    p["A"][p["m_indices"] < 0] = 0x38
+    got = bf16_to_f64(_grouped(ops, p))
+    _status_ok(ops)
+    assert np.all(got[p["m_indices"] < 0] == 0.0)
+    check_gemm(got, orc.gemm_grouped_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["m_indices"]), "grouped pad")
+
+
+def test_grouped_single_expert_equals_dense(ops):
+    p = inputs.grouped_fp8_problem(1, 384, 448, 512, seed=8, counts=[384])
+    Dg = _grouped(ops, p)
+    Dd = ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"][0]), to_dev(p["sfb"][0]))
+    _status_ok(ops)
+    assert torch.equal(Dg.view(torch.int16), Dd.view(torch.int16))
+
+
+def test_grouped_bad_index_is_flagged(ops):
+    p = inputs.grouped_fp8_problem(2, 256, 224, 256, seed=6, counts=[128, 128])
+    p["m_indices"][128] = 7  # block start names an expert that does not exist
+    _grouped(ops, p)
+    assert ops.device_status() == -7
+    _status_ok(ops)
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_wait_timeout_is_reported_and_context_survives(ops, orc):
+    # a 2 us wait limit cannot hold a K=8192 tile: a wait runs out, the kernel winds down
+    p = inputs.dense_fp8_problem(512, 448, 8192, seed=4)
+    args = [to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")]
+    old = ops.set_wait_timeout_ns(2000)
+    try:
+        ops.gemm_fp8_nt(*args)
+        assert ops.device_status() == -6
+    finally:
+        ops.set_wait_timeout_ns(old)
+    D = ops.gemm_fp8_nt(*args)
+    _status_ok(ops)
+    check_gemm(bf16_to_f64(D), orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"]), "after timeout")
