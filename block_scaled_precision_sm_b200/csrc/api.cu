@@ -10,6 +10,7 @@
 
 #include "bsp.h"
 #include "gemm.cuh"
+#include "internal.h"
 #include "sf_transform.cuh"
 
 namespace bsp {
@@ -146,7 +147,62 @@ int check_ld(int64_t ld, int64_t min_elems, int esize) {
         if (_rc != BSP_OK) return _rc; \
     } while (0)
 
+// Device facts without the per-device context (which allocates the status word).
+int device_facts_noalloc(int* sms) {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BSP_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return BSP_ERR_CUDA;
+    if (major != 10) return BSP_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return BSP_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return BSP_OK;
+}
+
 }  // namespace
+
+namespace detail {
+
+int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
+                           cudaStream_t stream) {
+    const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
+    if (grid.y > 65535u) return BSP_ERR_UNSUPPORTED;
+    sf_transform_kernel<1><<<grid, 256, 0, stream>>>(in, mn, kb, ld_in, static_cast<uint16_t*>(out), ld_out, status);
+    g_launches.fetch_add(1);
+    return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
+}
+
+int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
+                           int K, int64_t lda, int64_t ldb, int64_t ldd, int64_t ld_sfa, int64_t ld_sfb,
+                           int sfb_gran_n, int* status, cudaStream_t stream) {
+    DeviceCtx ctx;
+    BSP_TRY(device_facts_noalloc(&ctx.sms));
+    ctx.ready = true;
+    ctx.status = status;
+    const int kb = K / 128, words = (kb + 1) / 2;
+    const int mn_b = (N + sfb_gran_n - 1) / sfb_gran_n;
+    CUtensorMap ta, tb, tsa, tsb;
+    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, CfgFP8::BM));
+    BSP_TRY(operand_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, ldb, CfgFP8::BN));
+    BSP_TRY(sf_map(&tsa, sfa, M, words, ld_sfa, CfgFP8::BM, 1, 1));
+    BSP_TRY(sf_map(&tsb, sfb, mn_b, words, ld_sfb, sfb_gran_n == 1 ? CfgFP8::BN : 16, 1, 1));
+    GemmArgs a{};
+    a.M = M, a.N = N, a.K = K;
+    a.num_kb = kb;
+    a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
+    a.sfb_gran = sfb_gran_n;
+    return launch<CfgFP8>(ta, tb, tsa, tsb, a, ctx, stream);
+}
+
+}  // namespace detail
 }  // namespace bsp
 
 using namespace bsp;

@@ -1,0 +1,22 @@
+// internal.h — launch helpers shared between translation units of libbsp.so.  They take
+// the status word from the caller and never allocate device memory.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace bsp {
+namespace detail {
+
+// SF words from uint8 UE8M0 bytes [mn][ld_in] into int16 [ceil(kb/2)][ld_out]; faults latch `status`.
+int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
+                           cudaStream_t stream);
+
+// FP8 block-scaled GEMM on packed SF words, same rules as gemm_fp8_nt; faults latch `status`.
+int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
+                           int K, int64_t lda, int64_t ldb, int64_t ldd, int64_t ld_sfa, int64_t ld_sfb,
+                           int sfb_gran_n, int* status, cudaStream_t stream);
+
+}  // namespace detail
+}  // namespace bsp

@@ -130,6 +130,39 @@ int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t l
                        void* sf_out, int64_t ld_out, void* stream);
 
 /*
+ * gemm_fp8_nt_noalloc — the FP8 block-scaled GEMM of gemm_fp8_nt for callers that cannot
+ * allocate device memory.  (The pages have no counterpart; this is a deployment variant.)
+ *
+ * Who needs it: gemm_fp8_nt wants its scale factors already packed and keeps its status word
+ * in memory the library cudaMalloc's on first use.  A caller that holds plain UE8M0 bytes
+ * and cannot call cudaMalloc — for example code running under a framework whose caching
+ * allocator has already reserved the device memory, a loop that cannot afford cudaMalloc's
+ * implicit device synchronisation, or a C program that forbids allocation after start-up —
+ * would have nowhere to put the packed words.  This call packs them into a 4 MiB scratch
+ * array that the library defines statically on the device (every GPU that loads the library
+ * holds it until the process exits), then runs the same GEMM kernel.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *
+ *   A, B, D, M, N, K, lda, ldb, ldd, sfb_gran_n: as in gemm_fp8_nt.
+ *   sfa_e8m0  uint8 UE8M0 bytes [M][ld_sfa_in], one per row of A and 128 K (ld_sfa_in >= K/128).
+ *   sfb_e8m0  uint8 UE8M0 bytes [ceil(N/sfb_gran_n)][ld_sfb_in] (ld_sfb_in >= K/128).
+ *   status    device int, output: set to 0 by the call, then latched by its kernels like the
+ *             status word of the other calls (BSP_ERR_TIMEOUT, BSP_ERR_DEVICE_CHECK); read it
+ *             after the stream has finished.
+ * Limit: the packed words, round_up(M,8) + round_up(ceil(N/g),8) int16 per K pair (the SFA
+ * part rounded up to 256 bytes), must fit in 4 MiB — for example M up to about 32000 at
+ * K = 16384; larger calls return BSP_ERR_UNSUPPORTED and launch nothing.
+ * Every call shares the one scratch array and overwrites it: calls that overlap on the GPU
+ * (different streams, or different host threads on one device) race on it and must be
+ * ordered by the caller.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ * capture.
+ */
+int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const void* B, const void* sfb_e8m0, void* D,
+                        int* status, int M, int N, int K, int64_t lda, int64_t ldb, int64_t ldd,
+                        int64_t ld_sfa_in, int64_t ld_sfb_in, int sfb_gran_n, void* stream);
+
+/*
  * bsp_get_device_status — synchronises `stream`, then returns and clears the status
  * word latched by kernels on the current device (BSP_OK if nothing was latched).
  */
