@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only-headline", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "sf_transform"],
+                    help="launch only this kernel (warm-up + steps launches, no timing) for an ncu capture")
     return ap.parse_args()
 
 
@@ -475,9 +477,57 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """Only the named kernel, warm-up + steps times, at the workload's full size (for ncu)."""
+    import torch
+
+    from block_scaled_precision_sm_b200 import ops
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    if args.profile == "fp8":
+        p, dv = fp8_device_problem(torch, M, N, K, seed=100)
+        sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
+        D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # noqa: E731
+    elif args.profile == "bf16":
+        p = inputs.dense_bf16_problem(M, N, K, seed=2)
+        A = torch.from_numpy(p["A"]).cuda().view(torch.bfloat16)
+        B = torch.from_numpy(p["B"]).cuda().view(torch.bfloat16)
+        D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.gemm_bf16_nt(A, B, D)  # noqa: E731
+    elif args.profile == "fp4":
+        p = inputs.dense_fp4_problem(M, N, K, seed=6)
+        d4 = {key: torch.from_numpy(p[key]).cuda() for key in ("A", "sfa", "B", "sfb")}
+        sa, sb = ops.transform_sf_ue8m0(d4["sfa"]), ops.transform_sf_ue8m0(d4["sfb"])
+        D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.gemm_fp4_nt(d4["A"], sa, d4["B"], sb, D)  # noqa: E731
+    elif args.profile == "grouped":
+        g = inputs.grouped_fp8_problem(32, 32768, 4096, 7168, seed=8)
+        dg = {key: torch.from_numpy(g[key]).cuda() for key in ("A", "sfa", "B", "m_indices")}
+        sa = ops.transform_sf_ue8m0(dg["sfa"])
+        sb = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(g["sfb"][e]).cuda()) for e in range(32)])
+        D = torch.empty((g["M"], 4096), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.m_grouped_gemm_fp8_nt_contiguous(dg["A"], sa, dg["B"], sb, dg["m_indices"], D)  # noqa
+    else:
+        g = inputs.grouped_fp8_problem(32, 32768, 4096, 7168, seed=8)
+        s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()
+        w = torch.empty((28, ops.sf_ld(g["M"])), dtype=torch.int16, device="cuda")
+        fn = lambda: ops.transform_sf_ue8m0(s32, out=w)  # noqa: E731
+    torch.cuda.synchronize()
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    status = ops.device_status()
+    print(json.dumps({"profile": args.profile, "launches": args.warmup + args.steps, "status": status}))
+    if status != 0:
+        raise SystemExit(1)
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
