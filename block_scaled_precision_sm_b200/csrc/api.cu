@@ -11,7 +11,14 @@
 #include "bsp.h"
 #include "gemm.cuh"
 #include "internal.h"
+#include "sf_layout.cuh"
 #include "sf_transform.cuh"
+
+#define BSP_TRY(x)                     \
+    do {                               \
+        const int _rc = (x);           \
+        if (_rc != BSP_OK) return _rc; \
+    } while (0)
 
 namespace bsp {
 namespace {
@@ -96,44 +103,175 @@ int operand_map_3d(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t 
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Scale-word map: int16 [words][ld], box = box_mn x box_words; rank 3 ([groups][words][ld],
-// box depth 1) when `grouped`, since the grouped kernel issues 3-D loads even for one group.
-int sf_map(CUtensorMap* m, const void* base, int64_t mn, int64_t words, int64_t ld, int box_mn, int box_words,
-           int64_t groups, bool grouped = false) {
-    const cuuint64_t dims[3] = {(cuuint64_t)mn, (cuuint64_t)words, (cuuint64_t)groups};
-    const cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(ld * 2 * words)};
-    const cuuint32_t box[3] = {(cuuint32_t)box_mn, (cuuint32_t)box_words, 1};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, grouped ? 3 : 2, base, dims, strides, box,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 template <class C>
 int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
            GemmArgs a, const DeviceCtx& ctx, cudaStream_t stream) {
+    // D: bf16 [M][ldd], stored in 32 x 32 blocks through a 64-byte-swizzled staging buffer
+    CUtensorMap td;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
+        const cuuint64_t strides[1] = {(cuuint64_t)(a.ldd * 2)};
+        const cuuint32_t box[2] = {32, 32};
+        BSP_TRY(encode(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.D, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B));
+    }
     static std::once_flag attr_once[kMaxDevices];
+    static int max_workers[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     cudaError_t attr_err = cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C::CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     std::call_once(attr_once[dev], [&] {
         attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        int clusters = 0;
+        cfg.gridDim = dim3(C::CTAS * (ctx.sms / C::CTAS));
+        if (attr_err == cudaSuccess)
+            attr_err = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<C>, &cfg);
+        // a persistent grid larger than what is co-resident would serialise its last workers
+        max_workers[dev] = clusters > 0 ? clusters : ctx.sms / C::CTAS;
     });
     if (attr_err != cudaSuccess) return BSP_ERR_CUDA;
-    a.m_blocks = (a.M + C::BM - 1) / C::BM;
+    a.m_blocks = (a.M + C::TILE_M - 1) / C::TILE_M;
     a.n_blocks = (a.N + C::BN - 1) / C::BN;
     a.num_tiles = a.m_blocks * a.n_blocks;
     a.group_m = 16;
     a.status = ctx.status;
     a.timeout_ns = g_timeout_ns.load();
-    const int grid = a.num_tiles < ctx.sms ? a.num_tiles : ctx.sms;
-    gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ta, tb, tsa, tsb, a);
+    const int workers = a.num_tiles < max_workers[dev] ? a.num_tiles : max_workers[dev];
+    cfg.gridDim = dim3(C::CTAS * workers);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, td, a);
+    g_launches.fetch_add(1);
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? BSP_OK : BSP_ERR_CUDA;
+}
+
+//                       kind        BN   stages sf_stages grouped pair
+using CfgBF16P = GemmCfg<Kind::BF16, 224, 6, 1, false, true>;
+using CfgFP8P = GemmCfg<Kind::FP8, 224, 6, 3, false, true>;
+using CfgFP4P = GemmCfg<Kind::FP4, 224, 6, 6, false, true>;
+using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, 1, false, false>;
+using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, 2, false, false>;
+using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, 4, false, false>;
+using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, 2, true, false>;
+
+// Problem description shared by the GEMM entry points.
+struct Operands {
+    const void *A, *B, *sfa, *sfb;
+    int64_t lda, ldb, ld_sfa, ld_sfb;
+    int mn_b;         // scale rows of B (per expert)
+    int words;        // int16 scale words along K
+    int groups = 1;   // experts (grouped layout)
+};
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Scale chunks of config C: layouts of the A and B chunk tensors and their bytes.
+template <class C>
+struct ScaleChunks {
+    SfLayout a, b;
+    int64_t a_bytes = 0, b_bytes = 0;
+    ScaleChunks(const Operands& o, const GemmArgs& g) {
+        const int q = (o.words + 2 * C::UT_WORDS - 1) / (2 * C::UT_WORDS);
+        a = SfLayout{g.M, 1, o.words, o.ld_sfa, 0, C::BM, 1, C::UT_WORDS, (g.M + C::BM - 1) / C::BM, q, 1};
+        const int64_t b_gstride = (int64_t)o.words * o.ld_sfb;
+        b = SfLayout{g.N, g.sfb_gran, o.words, o.ld_sfb, b_gstride, C::BN, C::SFB_ATOMS, C::UT_WORDS,
+                     (g.N + C::BN - 1) / C::BN, q, o.groups};
+        a_bytes = round_up((int64_t)q * a.tiles * C::SFA_CHUNK, 256);
+        b_bytes = round_up((int64_t)q * b.tiles * C::SFB_CHUNK * o.groups, 256);
+    }
+    int64_t bytes() const { return a_bytes + b_bytes; }
+};
+
+int launch_sf_layout(const void* in_a, const SfLayout& pa, void* out_a, const void* in_b, const SfLayout& pb,
+                     void* out_b, cudaStream_t stream) {
+    const int64_t total = sf_layout_words(pa) + sf_layout_words(pb);
+    const int64_t blocks = (total + 255) / 256;
+    sf_tmem_layout_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(in_a), pa, static_cast<uint32_t*>(out_a), static_cast<const uint16_t*>(in_b),
+        pb, static_cast<uint32_t*>(out_b));
     g_launches.fetch_add(1);
     return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
 }
 
-using CfgBF16 = GemmCfg<Kind::BF16, 224, 5, false>;
-using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false>;
-using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false>;
-using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true>;
+// Stream-ordered scratch from a pool this library owns on each device, which keeps its memory
+// mapped between calls (the default pool would hand it back to the driver at every
+// synchronisation and map it again on the next call).
+int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSP_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (pools[dev] == nullptr) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if (cudaMemPoolCreate(&pools[dev], &props) != cudaSuccess) return BSP_ERR_CUDA;
+            uint64_t keep = UINT64_MAX;
+            if (cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+                return BSP_ERR_CUDA;
+        }
+    }
+    return cudaMallocFromPoolAsync(p, bytes, pools[dev], stream) == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
+}
+
+// Chunk tensor map: 8-byte elements, one chunk per (row tile, group [, expert]).
+int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int q, int experts_or_neg) {
+    // experts_or_neg < 0: a rank-4 map over -experts_or_neg experts (the grouped kernel's 4-D loads)
+    const int experts = experts_or_neg < 0 ? -experts_or_neg : experts_or_neg;
+    const cuuint64_t dims[4] = {(cuuint64_t)(chunk_bytes / 8), (cuuint64_t)tiles, (cuuint64_t)q,
+                                (cuuint64_t)experts};
+    const cuuint64_t strides[3] = {(cuuint64_t)chunk_bytes, (cuuint64_t)chunk_bytes * tiles,
+                                   (cuuint64_t)chunk_bytes * tiles * q};
+    const cuuint32_t box[4] = {(cuuint32_t)(chunk_bytes / 8), 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, experts_or_neg < 0 ? 4 : 3, base, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Encode the tensor maps for config C and launch it.  Scaled kinds first lay the scales out
+// as TMEM chunks in `ws` (stream-ordered scratch on the caller's stream when ws is null).
+template <class C>
+int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_t stream, void* ws = nullptr) {
+    constexpr bool bf16 = C::kind == Kind::BF16;
+    const auto dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const int es = bf16 ? 2 : 1;
+    const int64_t row_elems = C::kind == Kind::FP4 ? a.K / 2 : a.K;
+    CUtensorMap ta, tb, tsa, tsb;
+    BSP_TRY(operand_map(&ta, dt, es, o.A, row_elems, a.M, o.lda, C::BM));
+    if constexpr (C::GROUPED)
+        BSP_TRY(operand_map_3d(&tb, o.B, a.K, a.N, o.groups, C::BN_CTA));
+    else
+        BSP_TRY(operand_map(&tb, dt, es, o.B, row_elems, a.N, o.ldb, C::BN_CTA));
+    a.num_kb = (int)((row_elems * es + 127) / 128);
+    if constexpr (!C::SCALED) {
+        return launch<C>(ta, tb, ta, tb, a, ctx, stream);
+    } else {
+        const ScaleChunks<C> sc(o, a);
+        bool owned = false;
+        if (ws == nullptr) {
+            BSP_TRY(scratch_alloc(&ws, (size_t)sc.bytes(), stream));
+            owned = true;
+        }
+        char* wa = static_cast<char*>(ws);
+        char* wb = wa + sc.a_bytes;
+        int rc = launch_sf_layout(o.sfa, sc.a, wa, o.sfb, sc.b, wb, stream);
+        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, sc.a.tiles, sc.a.q, 1);
+        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, sc.b.tiles, sc.b.q, C::GROUPED ? -o.groups : 1);
+        if (rc == BSP_OK) rc = launch<C>(ta, tb, tsa, tsb, a, ctx, stream);
+        if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && rc == BSP_OK) rc = BSP_ERR_CUDA;
+        return rc;
+    }
+}
 
 int check_ld(int64_t ld, int64_t min_elems, int esize) {
     if (ld < min_elems) return BSP_ERR_SHAPE;
@@ -141,11 +279,6 @@ int check_ld(int64_t ld, int64_t min_elems, int esize) {
     return BSP_OK;
 }
 
-#define BSP_TRY(x)                     \
-    do {                               \
-        const int _rc = (x);           \
-        if (_rc != BSP_OK) return _rc; \
-    } while (0)
 
 // Device facts without the per-device context (which allocates the status word).
 int device_facts_noalloc(int* sms) {
@@ -180,26 +313,30 @@ int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* 
     return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
 }
 
+int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
+    const int kb = K / 128, words = (kb + 1) / 2;
+    const Operands o{nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, (N + sfb_gran_n - 1) / sfb_gran_n, words};
+    GemmArgs a{};
+    a.M = M, a.N = N, a.K = K, a.sfb_gran = sfb_gran_n;
+    return M > 128 ? ScaleChunks<CfgFP8P>(o, a).bytes() : ScaleChunks<CfgFP8>(o, a).bytes();
+}
+
 int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
                            int K, int64_t lda, int64_t ldb, int64_t ldd, int64_t ld_sfa, int64_t ld_sfb,
-                           int sfb_gran_n, int* status, cudaStream_t stream) {
+                           int sfb_gran_n, int* status, void* scale_scratch, cudaStream_t stream) {
     DeviceCtx ctx;
     BSP_TRY(device_facts_noalloc(&ctx.sms));
     ctx.ready = true;
     ctx.status = status;
     const int kb = K / 128, words = (kb + 1) / 2;
     const int mn_b = (N + sfb_gran_n - 1) / sfb_gran_n;
-    CUtensorMap ta, tb, tsa, tsb;
-    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, CfgFP8::BM));
-    BSP_TRY(operand_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, ldb, CfgFP8::BN));
-    BSP_TRY(sf_map(&tsa, sfa, M, words, ld_sfa, CfgFP8::BM, 1, 1));
-    BSP_TRY(sf_map(&tsb, sfb, mn_b, words, ld_sfb, sfb_gran_n == 1 ? CfgFP8::BN : 16, 1, 1));
+    const Operands o{A, B, sfa, sfb, lda, ldb, ld_sfa, ld_sfb, mn_b, words};
     GemmArgs a{};
     a.M = M, a.N = N, a.K = K;
-    a.num_kb = kb;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    return launch<CfgFP8>(ta, tb, tsa, tsb, a, ctx, stream);
+    return M > 128 ? launch_gemm<CfgFP8P>(o, a, ctx, stream, scale_scratch)
+                   : launch_gemm<CfgFP8>(o, a, ctx, stream, scale_scratch);
 }
 
 }  // namespace detail
@@ -219,15 +356,13 @@ int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K, int
     BSP_TRY(check_ld(ldd, N, 2));
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
-    CUtensorMap ta, tb;
-    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, lda, CfgBF16::BM));
-    BSP_TRY(operand_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, K, N, ldb, CfgBF16::BN));
+    const Operands o{A, B, nullptr, nullptr, lda, ldb, 0, 0, 0, 0};
     GemmArgs a{};
     a.M = M, a.N = N, a.K = K;
-    a.num_kb = (K + 63) / 64;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
-    return launch<CfgBF16>(ta, tb, ta, tb, a, *ctx, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return M > 128 ? launch_gemm<CfgBF16P>(o, a, *ctx, st) : launch_gemm<CfgBF16>(o, a, *ctx, st);
 }
 
 int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N, int K,
@@ -246,17 +381,13 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     BSP_TRY(check_ld(ld_sfb, mn_b, 2));
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
-    CUtensorMap ta, tb, tsa, tsb;
-    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, lda, CfgFP8::BM));
-    BSP_TRY(operand_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, ldb, CfgFP8::BN));
-    BSP_TRY(sf_map(&tsa, sfa, M, words, ld_sfa, CfgFP8::BM, 1, 1));
-    BSP_TRY(sf_map(&tsb, sfb, mn_b, words, ld_sfb, sfb_gran_n == 1 ? CfgFP8::BN : 16, 1, 1));
+    const Operands o{A, B, sfa, sfb, lda, ldb, ld_sfa, ld_sfb, mn_b, words};
     GemmArgs a{};
     a.M = M, a.N = N, a.K = K;
-    a.num_kb = kb;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    return launch<CfgFP8>(ta, tb, tsa, tsb, a, *ctx, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return M > 128 ? launch_gemm<CfgFP8P>(o, a, *ctx, st) : launch_gemm<CfgFP8>(o, a, *ctx, st);
 }
 
 int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N, int K,
@@ -264,7 +395,7 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     if (!A || !sfa || !B || !sfb || !D || M <= 0 || N <= 0 || K <= 0) return BSP_ERR_ARG;
     if (K % 64) return BSP_ERR_SHAPE;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned16(sfb)) return BSP_ERR_ALIGN;
-    const int kb = K / 32, words = kb / 2;
+    const int words = K / 64;
     BSP_TRY(check_ld(lda, K / 2, 1));
     BSP_TRY(check_ld(ldb, K / 2, 1));
     BSP_TRY(check_ld(ldd, N, 2));
@@ -272,17 +403,13 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     BSP_TRY(check_ld(ld_sfb, N, 2));
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
-    CUtensorMap ta, tb, tsa, tsb;
-    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K / 2, M, lda, CfgFP4::BM));
-    BSP_TRY(operand_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K / 2, N, ldb, CfgFP4::BN));
-    BSP_TRY(sf_map(&tsa, sfa, M, words, ld_sfa, CfgFP4::BM, 4, 1));
-    BSP_TRY(sf_map(&tsb, sfb, N, words, ld_sfb, CfgFP4::BN, 4, 1));
+    const Operands o{A, B, sfa, sfb, lda, ldb, ld_sfa, ld_sfb, N, words};
     GemmArgs a{};
     a.M = M, a.N = N, a.K = K;
-    a.num_kb = (K / 2 + 127) / 128;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
-    return launch<CfgFP4>(ta, tb, tsa, tsb, a, *ctx, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return M > 128 ? launch_gemm<CfgFP4P>(o, a, *ctx, st) : launch_gemm<CfgFP4>(o, a, *ctx, st);
 }
 
 int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void* B, const void* sfb, void* D,
@@ -301,18 +428,14 @@ int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void*
     BSP_TRY(check_ld(ld_sfb, mn_b, 2));
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
-    CUtensorMap ta, tb, tsa, tsb;
-    BSP_TRY(operand_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M_total, K, CfgGrouped::BM));
-    BSP_TRY(operand_map_3d(&tb, B, K, N, G, CfgGrouped::BN));
-    BSP_TRY(sf_map(&tsa, sfa, M_total, words, ld_sfa, CfgGrouped::BM, 1, 1));
-    BSP_TRY(sf_map(&tsb, sfb, mn_b, words, ld_sfb, sfb_gran_n == 1 ? CfgGrouped::BN : 16, 1, G, true));
+    Operands o{A, B, sfa, sfb, K, K, ld_sfa, ld_sfb, mn_b, words};
+    o.groups = G;
     GemmArgs a{};
     a.M = M_total, a.N = N, a.K = K;
-    a.num_kb = kb;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = N;
     a.m_indices = m_indices, a.G = G;
     a.sfb_gran = sfb_gran_n;
-    return launch<CfgGrouped>(ta, tb, tsa, tsb, a, *ctx, static_cast<cudaStream_t>(stream));
+    return launch_gemm<CfgGrouped>(o, a, *ctx, static_cast<cudaStream_t>(stream));
 }
 
 int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in, void* sf_out, int64_t ld_out,

@@ -5,19 +5,34 @@
 // Pipeline (the pages' "operand reuse and pipelining" with staged buffers and ready
 // signals, "DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Reúso de
 // operandos e pipelining na prática", rebuilt for Blackwell):
-//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and the packed int16 scale
-//               words of each K step into an S-stage shared-memory ring; "full" mbarrier
-//               per stage (transaction-counted).
-//   warp 1      owns tensor memory (TMEM); per stage it rewrites the MN-major scale
-//               words into the 32-row x 16-byte layout the scale copy expects, copies
-//               them into TMEM (tcgen05.cp) and issues the tcgen05.mma instructions
-//               (one elected lane), then commits to the stage's "empty" mbarrier.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in TMEM so
-//               the next tile's MMAs overlap), round to bf16, store to D.
-// Tiles: 128 x BLOCK_N output tiles, one CTA per SM walking tiles in a grouped raster.
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle) into an S-stage shared-memory
+//               ring ("full"/"empty" mbarriers, transaction-counted), and every SF_PERIOD K
+//               steps one chunk of scale words per operand into a small ring ("sf_full" /
+//               "sf_empty").  The chunks were laid out beforehand (sf_layout.cuh) exactly as
+//               the scale copy reads them, so no thread rearranges scales on chip.
+//   warp 1      owns TMEM; in the MMA-issuing CTA one elected lane issues tcgen05.cp of each
+//               scale chunk into a rotating TMEM slot and the tcgen05.mma instructions,
+//               committing to the "empty" / "sf_empty" barriers.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in TMEM so the
+//               next tile's MMAs overlap), round to bf16, stage 32 x 32 blocks in a swizzled
+//               shared-memory buffer (two per warp) and TMA-store them to D.
+//
+// PAIR = true: a cluster of two CTAs computes a 256 x BN tile with cta_group::2 MMAs.  CTA r
+// loads A rows [128r, 128r+128) and B rows [r*BN/2, (r+1)*BN/2) of the tile into its own
+// shared memory (each SM streams half of B: operand reuse across the pair without
+// multicast) plus its own scale chunks (its 128 A rows, all BN B rows), the leader CTA
+// (rank 0) issues the MMAs and the scale copies, and the accumulator rows of CTA r land in
+// its own TMEM.  All loads signal the leader's barriers; the leader's commits are multicast
+// to both CTAs' barriers; the peer's epilogue arrives on the leader's barrier remotely.
+//
+// FP8 scales are one byte per (row, 128 K): a scale group of four K steps is one 32-bit word
+// per row and the MMA of K step kb selects byte kb % 4.  FP4 scales are one byte per (row,
+// 32 K): a group is one K step of 256, two words per row, and an MMA (K = 64) selects a byte
+// pair.
+//
 // Every wait is bounded: past the deadline the CTA latches BSP_ERR_TIMEOUT in the status
-// word, raises a shared abort flag, drains its own in-flight copies and MMAs, frees TMEM
-// and returns.
+// word, raises a shared abort flag, drains its own in-flight copies and MMAs, frees TMEM and
+// returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,7 +49,7 @@ constexpr int kStatusDeviceCheck = -7;  // BSP_ERR_DEVICE_CHECK
 struct GemmArgs {
     int M, N, K;
     int num_kb;    // K steps of 128 bytes per row
-    int m_blocks;  // ceil(M / 128)
+    int m_blocks;  // ceil(M / tile rows)
     int n_blocks;  // ceil(N / BLOCK_N)
     int num_tiles;
     int group_m;   // raster: m-blocks per group
@@ -47,30 +62,34 @@ struct GemmArgs {
     unsigned long long timeout_ns;
 };
 
-template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_>
+template <Kind KIND, int BLOCK_N_, int STAGES_, int SF_STAGES_, bool GROUPED_, bool PAIR_>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
-    static constexpr int BM = 128;
-    static constexpr int BN = BLOCK_N_;
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int BM = 128;              // A / D rows per CTA
+    static constexpr int TILE_M = BM * CTAS;    // rows per tile
+    static constexpr int BN = BLOCK_N_;         // columns per tile
+    static constexpr int BN_CTA = BN / CTAS;    // B rows loaded per CTA
     static constexpr int STAGES = STAGES_;
+    static constexpr int SF_STAGES = SF_STAGES_;
     static constexpr bool GROUPED = GROUPED_;
     static constexpr bool SCALED = KIND != Kind::BF16;
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BLOCK_N");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && BN_CTA % 8 == 0, "BLOCK_N");
 
     // One K step = one 128-byte swizzle row per operand row: 64 bf16, 128 E4M3, 256 E2M1.
     static constexpr int A_BYTES = BM * 128;
-    static constexpr int B_BYTES = BN * 128;
-    // int16 scale words per row per K step: FP8 one (the word covers two 128-K blocks,
-    // the step uses one byte of it); FP4 four (8 blocks of 32 K).
-    static constexpr int SF_WORDS = KIND == Kind::FP4 ? 4 : 1;
-    // 32-bit TMEM scale words per row per K step.
-    static constexpr int UT_WORDS = KIND == Kind::FP4 ? 2 : 1;
-    static constexpr int SFB_ATOMS = (BN + 127) / 128;
-    static constexpr int SFA_RAW = SCALED ? ((BM * SF_WORDS * 2 + 127) / 128) * 128 : 0;
-    static constexpr int SFB_RAW = SCALED ? (((BN > 16 ? BN : 16) * SF_WORDS * 2 + 127) / 128) * 128 : 0;
-    static constexpr int UTA_BYTES = SCALED ? UT_WORDS * 512 : 0;
-    static constexpr int UTB_BYTES = SCALED ? UT_WORDS * SFB_ATOMS * 512 : 0;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_RAW + SFB_RAW + UTA_BYTES + UTB_BYTES;
+    static constexpr int B_BYTES = BN_CTA * 128;
+    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment");
+
+    // Scale groups: every SF_PERIOD K steps, UT_WORDS 32-bit TMEM words per row; a chunk per
+    // 128-row atom and word is 32 rows x 16 bytes.
+    static constexpr int SF_PERIOD = KIND == Kind::FP8 ? 4 : 1;
+    static constexpr int UT_WORDS = KIND == Kind::FP8 ? 1 : 2;
+    static constexpr int SFB_ATOMS = (BN + 127) / 128;  // every CTA holds the scales of all BN rows
+    static constexpr int SFA_CHUNK = SCALED ? UT_WORDS * 512 : 0;
+    static constexpr int SFB_CHUNK = SCALED ? SFB_ATOMS * UT_WORDS * 512 : 0;
+    static constexpr int SF_STAGE_BYTES = SFA_CHUNK + SFB_CHUNK;
 
     // Tensor memory: two fp32 accumulators of BN columns, then rotating scale slots.
     static constexpr int TMEM_COLS = 512;
@@ -85,15 +104,16 @@ struct GemmCfg {
     // Shared memory map (offsets from a 1024-byte aligned base).
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_RAW;
-    static constexpr int OFF_UTA = OFF_SFB + STAGES * SFB_RAW;
-    static constexpr int OFF_UTB = OFF_UTA + STAGES * UTA_BYTES;
-    static constexpr int OFF_BAR = ((OFF_UTB + STAGES * UTB_BYTES + 7) / 8) * 8;
-    static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
+    // epilogue staging: per epilogue warp two 32 x 32 bf16 blocks (64-byte swizzle)
+    static constexpr int EPI_BLOCK = 32 * 32 * 2;
+    static constexpr int OFF_EPI = ((OFF_SF + (SCALED ? SF_STAGES * SF_STAGE_BYTES : 0) + 1023) / 1024) * 1024;
+    // full, empty [STAGES]; sf_full, sf_empty [SF_STAGES]; tmem_full, tmem_empty [2]; drain
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_STAGES + 5;
+    static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-    static_assert(B_BYTES % 1024 == 0, "B tile must keep 1024-byte alignment");
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
     static constexpr int THREADS = 192;
 };
@@ -117,13 +137,15 @@ __device__ __forceinline__ void latch_status(int* status, int code) {
 
 // Bounded wait on a phase of `bar`.  False if the deadline passed (status latched and
 // abort raised) or another role already aborted.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, const GemmArgs& a,
                                              volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto try_once = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (try_once()) return true;
     // try_wait itself suspends for a while before reporting "not yet", so the deadline and
     // the abort flag are checked after every failed try.
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!try_once()) {
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > a.timeout_ns) {
             latch_status(a.status, kStatusTimeout);
@@ -151,9 +173,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
 
 // Whole-warp wait: every lane waits, and the outcome is voted so the warp stays converged
 // (a lane that timed out takes all lanes with it).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const GemmArgs& a,
                                           volatile int* abort_flag) {
-    const bool ok = bounded_wait(bar, parity, a, abort_flag);
+    const bool ok = bounded_wait<CLUSTER>(bar, parity, a, abort_flag);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -161,29 +184,40 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
-                const GemmArgs args) {
+                const __grid_constant__ CUtensorMap tm_d, const GemmArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bars;
-    uint64_t* empty = bars + C::STAGES;
-    uint64_t* tmem_full = bars + 2 * C::STAGES;
-    uint64_t* tmem_empty = bars + 2 * C::STAGES + 2;
-    uint64_t* drain = bars + 2 * C::STAGES + 4;
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* sf_full = empty + C::STAGES;
+    uint64_t* sf_empty = sf_full + C::SF_STAGES;
+    uint64_t* tmem_full = sf_empty + C::SF_STAGES;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint64_t* drain = tmem_empty + 2;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x / 32;
     const uint32_t lane = threadIdx.x % 32;
+    const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int worker = blockIdx.x / C::CTAS;
+    const int workers = gridDim.x / C::CTAS;
+    constexpr uint16_t kPairMask = 0x3;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int j = 0; j < C::SF_STAGES; ++j) {
+            mbar_init(&sf_full[j], 1);
+            mbar_init(&sf_empty[j], 1);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full[b], 1);
-            mbar_init(&tmem_empty[b], 4);
+            mbar_init(&tmem_empty[b], 4 * C::CTAS);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -192,29 +226,39 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&tm_d);
         if constexpr (C::SCALED) {
             tma_prefetch_desc(&tm_sfa);
             tma_prefetch_desc(&tm_sfb);
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (C::PAIR) {
+            tmem_alloc_pair(tmem_base_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_base_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (C::PAIR)
+        cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t it = 0;
+            uint32_t it = 0, git = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+            for (int t = worker; t < args.num_tiles && ok; t += workers) {
                 const Tile tl = tile_of(args, t);
-                const int m0 = tl.m_blk * C::BM;
+                const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
                 const int n0 = tl.n_blk * C::BN;
+                const int nb0 = n0 + (int)rank * C::BN_CTA;
                 int g = 0;
                 if constexpr (C::GROUPED) {
                     g = __ldg(args.m_indices + m0);
@@ -224,61 +268,123 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
                 for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+                    if constexpr (C::SCALED) {
+                        if (kb % C::SF_PERIOD == 0) {
+                            const uint32_t j = git % C::SF_STAGES, jph = (git / C::SF_STAGES) & 1u;
+                            if (!bounded_wait(&sf_empty[j], jph ^ 1u, args, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            if (leader) mbar_arrive_expect_tx(&sf_full[j], C::CTAS * C::SF_STAGE_BYTES);
+                            uint8_t* sf = smem + C::OFF_SF + j * C::SF_STAGE_BYTES;
+                            const int q = kb / C::SF_PERIOD;
+                            // chunk coordinates: (0, row tile, group [, expert])
+                            if constexpr (C::PAIR) {
+                                const uint32_t lead_sf = mapa_shared(smem_u32(&sf_full[j]), 0);
+                                tma_load_3d_pair(sf, &tm_sfa, lead_sf, 0, m0 / C::BM, q);
+                                tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_sf, 0, tl.n_blk, q);
+                            } else {
+                                tma_load_3d(sf, &tm_sfa, &sf_full[j], 0, m0 / C::BM, q);
+                                if constexpr (C::GROUPED)
+                                    tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &sf_full[j], 0, tl.n_blk, q, g);
+                                else
+                                    tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &sf_full[j], 0, tl.n_blk, q);
+                            }
+                            ++git;
+                        }
+                    }
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!bounded_wait(&empty[s], ph ^ 1u, args, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    uint32_t bytes = C::A_BYTES + C::B_BYTES;
-                    if constexpr (C::SCALED)
-                        bytes += C::BM * C::SF_WORDS * 2 +
-                                 (args.sfb_gran == 1 ? C::BN * C::SF_WORDS * 2 : 16 * 2);
-                    mbar_arrive_expect_tx(&full[s], bytes);
+                    if (leader) mbar_arrive_expect_tx(&full[s], C::CTAS * (C::A_BYTES + C::B_BYTES));
                     uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
                     uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
-                    tma_load_2d(sa, &tm_a, &full[s], kx, m0);
-                    if constexpr (C::GROUPED)
-                        tma_load_3d(sb, &tm_b, &full[s], kx, n0, g);
-                    else
-                        tma_load_2d(sb, &tm_b, &full[s], kx, n0);
-                    if constexpr (C::SCALED) {
-                        // word row of this step: FP8 uses word kb/2 (byte kb%2); FP4 words 4kb..4kb+3
-                        const int wy = C::kind == Kind::FP4 ? kb * 4 : kb / 2;
-                        uint8_t* rsa = smem + C::OFF_SFA + s * C::SFA_RAW;
-                        uint8_t* rsb = smem + C::OFF_SFB + s * C::SFB_RAW;
-                        tma_load_2d(rsa, &tm_sfa, &full[s], m0, wy);
-                        const int bx = args.sfb_gran == 1 ? n0 : ((n0 / 128) & ~7);
+                    if constexpr (C::PAIR) {
+                        const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), 0);
+                        tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
+                        tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
+                    } else {
+                        tma_load_2d(sa, &tm_a, &full[s], kx, m0);
                         if constexpr (C::GROUPED)
-                            tma_load_3d(rsb, &tm_sfb, &full[s], bx, wy, g);
+                            tma_load_3d(sb, &tm_b, &full[s], kx, nb0, g);
                         else
-                            tma_load_2d(rsb, &tm_sfb, &full[s], bx, wy);
+                            tma_load_2d(sb, &tm_b, &full[s], kx, nb0);
                     }
                 }
             }
             // Wind down: wait (bounded) until the copies issued for the last stages landed.
-            const uint32_t last = it < (uint32_t)C::STAGES ? it : (uint32_t)C::STAGES;
-            for (uint32_t j = it - last; j < it; ++j) drain_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, args);
+            if (leader) {
+                const uint32_t last = it < (uint32_t)C::STAGES ? it : (uint32_t)C::STAGES;
+                for (uint32_t j = it - last; j < it; ++j)
+                    drain_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, args);
+                const uint32_t slast = git < (uint32_t)C::SF_STAGES ? git : (uint32_t)C::SF_STAGES;
+                for (uint32_t j = git - slast; j < git; ++j)
+                    drain_wait(&sf_full[j % C::SF_STAGES], (j / C::SF_STAGES) & 1u, args);
+            }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ scale staging + MMA
-        uint32_t it = 0, lt = 0;
+    } else if (warp == 1 && leader) {
+        // ------------------------------------------------------------ MMA issue
+        uint32_t it = 0, lt = 0, git = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x, ++lt) {
-            const Tile tl = tile_of(args, t);
-            const int n0 = tl.n_blk * C::BN;
+        for (int t = worker; t < args.num_tiles && ok; t += workers, ++lt) {
             const uint32_t buf = lt & 1u;
             const uint32_t aph = (lt >> 1) & 1u;
-            if (!warp_wait(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
+            if (!warp_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + buf * C::BN;
+            uint32_t slot = 0;
             for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+                if constexpr (C::SCALED) {
+                    if (kb % C::SF_PERIOD == 0) {
+                        // copy this group's scale chunks into TMEM slot git % SF_SLOTS
+                        const uint32_t j = git % C::SF_STAGES, jph = (git / C::SF_STAGES) & 1u;
+                        if (!warp_wait(&sf_full[j], jph, args, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        slot = git % C::SF_SLOTS;
+                        if (lane == 0) {
+                            const uint32_t sfa_col = C::ACC_COLS + slot * C::SF_SLOT_COLS;
+                            const uint32_t sfb_col = sfa_col + C::SFA_COLS;
+                            const uint8_t* ua = smem + C::OFF_SF + j * C::SF_STAGE_BYTES;
+                            const uint8_t* ub = ua + C::SFA_CHUNK;
+#pragma unroll
+                            for (int u = 0; u < C::UT_WORDS; ++u) {
+                                if constexpr (C::PAIR)
+                                    tc_cp_32x128b_warpx4_pair(tmem_base + sfa_col + 4 * u,
+                                                              smem_desc_rows16(ua + u * 512));
+                                else
+                                    tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(ua + u * 512));
+#pragma unroll
+                                for (int at = 0; at < C::SFB_ATOMS; ++at) {
+                                    const uint32_t col = tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at);
+                                    const uint64_t d = smem_desc_rows16(ub + (at * C::UT_WORDS + u) * 512);
+                                    if constexpr (C::PAIR)
+                                        tc_cp_32x128b_warpx4_pair(col, d);
+                                    else
+                                        tc_cp_32x128b_warpx4(col, d);
+                                }
+                            }
+                            // the chunk buffers are free once these copies completed
+                            if constexpr (C::PAIR)
+                                tc_commit_pair_mc(&sf_empty[j], kPairMask);
+                            else
+                                tc_commit(&sf_empty[j]);
+                        }
+                        __syncwarp();
+                        ++git;
+                    }
+                }
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1u;
                 if (!warp_wait(&full[s], ph, args, abort_flag)) {
@@ -286,74 +392,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t slot = it % C::SF_SLOTS;
-                const uint32_t sfa_col = C::ACC_COLS + slot * C::SF_SLOT_COLS;
-                const uint32_t sfb_col = sfa_col + C::SFA_COLS;
-                if constexpr (C::SCALED) {
-                    // MN-major int16 words -> rows of 16 bytes: row l holds the 32-bit words of
-                    // matrix rows l, l+32, l+64, l+96 (the layout the 32x128b scale copy reads).
-                    const uint16_t* rsa = reinterpret_cast<const uint16_t*>(smem + C::OFF_SFA + s * C::SFA_RAW);
-                    const uint16_t* rsb = reinterpret_cast<const uint16_t*>(smem + C::OFF_SFB + s * C::SFB_RAW);
-                    uint4* uta = reinterpret_cast<uint4*>(smem + C::OFF_UTA + s * C::UTA_BYTES);
-                    uint4* utb = reinterpret_cast<uint4*>(smem + C::OFF_UTB + s * C::UTB_BYTES);
-                    if constexpr (C::kind == Kind::FP8) {
-                        uta[lane] = make_uint4(rsa[lane], rsa[lane + 32], rsa[lane + 64], rsa[lane + 96]);
-                        const int x0 = (n0 / 128) & ~7;
-#pragma unroll
-                        for (int at = 0; at < C::SFB_ATOMS; ++at) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int r = at * 128 + c * 32 + (int)lane;
-                                uint32_t v = 0;
-                                if (r < C::BN) v = args.sfb_gran == 1 ? rsb[r] : rsb[(n0 + r) / 128 - x0];
-                                w[c] = v;
-                            }
-                            utb[at * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    } else {  // FP4: word u of a row packs int16 words 2u (low half) and 2u+1
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int r = c * 32 + (int)lane;
-                                w[c] = (uint32_t)rsa[(2 * u) * C::BM + r] | ((uint32_t)rsa[(2 * u + 1) * C::BM + r] << 16);
-                            }
-                            uta[u * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-#pragma unroll
-                            for (int at = 0; at < C::SFB_ATOMS; ++at) {
-#pragma unroll
-                                for (int c = 0; c < 4; ++c) {
-                                    const int r = at * 128 + c * 32 + (int)lane;
-                                    w[c] = r < C::BN ? ((uint32_t)rsb[(2 * u) * C::BN + r] |
-                                                        ((uint32_t)rsb[(2 * u + 1) * C::BN + r] << 16))
-                                                     : 0u;
-                                }
-                                utb[(u * C::SFB_ATOMS + at) * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
-                            }
-                        }
-                    }
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
                 if (lane == 0) {
-                    const uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
-                    const uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-                    const uint64_t adesc = smem_desc_k_sw128(sa);
-                    const uint64_t bdesc = smem_desc_k_sw128(sb);
-                    if constexpr (C::SCALED) {
-                        const uint8_t* uta = smem + C::OFF_UTA + s * C::UTA_BYTES;
-                        const uint8_t* utb = smem + C::OFF_UTB + s * C::UTB_BYTES;
-#pragma unroll
-                        for (int u = 0; u < C::UT_WORDS; ++u) {
-                            tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(uta + u * 512));
-#pragma unroll
-                            for (int at = 0; at < C::SFB_ATOMS; ++at)
-                                tc_cp_32x128b_warpx4(tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at),
-                                                     smem_desc_rows16(utb + (u * C::SFB_ATOMS + at) * 512));
-                        }
-                    }
+                    const uint64_t adesc = smem_desc_k_sw128(smem + C::OFF_A + s * C::A_BYTES);
+                    const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + s * C::B_BYTES);
+                    const uint32_t sfa_t = tmem_base + C::ACC_COLS + slot * C::SF_SLOT_COLS;
+                    const uint32_t sfb_t = sfa_t + C::SFA_COLS;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         // 32 bytes of K per MMA: 16 bf16, 32 E4M3, 64 E2M1
@@ -361,39 +404,62 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         const uint64_t bd = bdesc + (uint64_t)(2 * i);
                         const uint32_t acc = (kb > 0 || i > 0) ? 1u : 0u;
                         if constexpr (C::kind == Kind::BF16) {
-                            tc_mma_f16(d_tmem, ad, bd, idesc_bf16(C::BM, C::BN), acc);
+                            const uint32_t id = idesc_bf16(C::TILE_M, C::BN);
+                            if constexpr (C::PAIR)
+                                tc_mma_f16_pair(d_tmem, ad, bd, id, acc);
+                            else
+                                tc_mma_f16(d_tmem, ad, bd, id, acc);
                         } else if constexpr (C::kind == Kind::FP8) {
-                            const uint32_t id = (uint32_t)(kb & 1);
-                            tc_mma_mxf8(d_tmem, ad, bd, idesc_block_scaled(C::BM, C::BN, 0u, id, id),
-                                        tmem_base + sfa_col, tmem_base + sfb_col, acc);
+                            const uint32_t sid = (uint32_t)(kb % 4);
+                            const uint32_t id = idesc_block_scaled(C::TILE_M, C::BN, 0u, sid, sid);
+                            if constexpr (C::PAIR)
+                                tc_mma_mxf8_pair(d_tmem, ad, bd, id, sfa_t, sfb_t, acc);
+                            else
+                                tc_mma_mxf8(d_tmem, ad, bd, id, sfa_t, sfb_t, acc);
                         } else {
-                            const uint32_t u = (uint32_t)(i >> 1), id = (uint32_t)((i & 1) * 2);
-                            tc_mma_mxf4(d_tmem, ad, bd, idesc_block_scaled(C::BM, C::BN, 1u, id, id),
-                                        tmem_base + sfa_col + 4 * u, tmem_base + sfb_col + 4 * C::SFB_ATOMS * u,
-                                        acc);
+                            const uint32_t u = (uint32_t)(i >> 1), sid = (uint32_t)((i & 1) * 2);
+                            const uint32_t id = idesc_block_scaled(C::TILE_M, C::BN, 1u, sid, sid);
+                            if constexpr (C::PAIR)
+                                tc_mma_mxf4_pair(d_tmem, ad, bd, id, sfa_t + 4 * u, sfb_t + 4 * C::SFB_ATOMS * u, acc);
+                            else
+                                tc_mma_mxf4(d_tmem, ad, bd, id, sfa_t + 4 * u, sfb_t + 4 * C::SFB_ATOMS * u, acc);
                         }
                     }
-                    tc_commit(&empty[s]);
+                    if constexpr (C::PAIR)
+                        tc_commit_pair_mc(&empty[s], kPairMask);
+                    else
+                        tc_commit(&empty[s]);
                 }
                 __syncwarp();
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(&tmem_full[buf]);
+            if (lane == 0) {
+                if constexpr (C::PAIR)
+                    tc_commit_pair_mc(&tmem_full[buf], kPairMask);
+                else
+                    tc_commit(&tmem_full[buf]);
+            }
             __syncwarp();
         }
         // Wind down: every MMA and scale copy this warp issued has completed.
         if (lane == 0) {
-            tc_commit(drain);
+            if constexpr (C::PAIR)
+                tc_commit_pair(drain);
+            else
+                tc_commit(drain);
             drain_wait(drain, 0, args);
         }
         __syncwarp();
+    } else if (warp == 1) {
+        // peer CTA of a pair: the leader issues every tensor-core instruction
     } else {
         // ------------------------------------------------------------ epilogue
         const uint32_t quarter = warp % 4;  // TMEM lanes this warp may read
-        uint32_t lt = 0;
-        for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++lt) {
+        uint8_t* epi = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BLOCK;
+        uint32_t lt = 0, nblk = 0;
+        for (int t = worker; t < args.num_tiles; t += workers, ++lt) {
             const Tile tl = tile_of(args, t);
-            const int m0 = tl.m_blk * C::BM;
+            const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
             const int n0 = tl.n_blk * C::BN;
             const uint32_t buf = lt & 1u;
             const uint32_t aph = (lt >> 1) & 1u;
@@ -409,46 +475,62 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (gi != g0 && gi != -1) latch_status(args.status, kStatusDeviceCheck);
                 }
             }
-            __nv_bfloat16* drow = args.D + (int64_t)row * args.ldd;
             const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + buf * C::BN;
 #pragma unroll 1
-            for (int c = 0; c < C::BN / 32; ++c) {
+            for (int c = 0; c < C::BN / 32; ++c, ++nblk) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(taddr + c * 32, r);
                 tmem_ld_wait();
                 if (c == C::BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+                    if (lane == 0) {
+                        if (leader)
+                            mbar_arrive(&tmem_empty[buf]);
+                        else
+                            mbar_arrive_remote(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
+                    }
                 }
-                if (row >= args.M) continue;
-                const int col0 = n0 + c * 32;
-                uint32_t packed[16];
+                // the store issued from this buffer two blocks ago has finished reading it
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint8_t* blk = epi + (nblk & 1u) * C::EPI_BLOCK;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 h = __float22bfloat162_rn(
-                        make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])));
-                    packed[j] = zero_row ? 0u : *reinterpret_cast<uint32_t*>(&h);
+                for (int q = 0; q < 4; ++q) {  // 16-byte chunk q of this row (8 columns)
+                    uint32_t w[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        __nv_bfloat162 v = __float22bfloat162_rn(make_float2(__uint_as_float(r[8 * q + 2 * h]),
+                                                                             __uint_as_float(r[8 * q + 2 * h + 1])));
+                        w[h] = zero_row ? 0u : *reinterpret_cast<uint32_t*>(&v);
+                    }
+                    // 64-byte swizzle: chunk q of row l sits at chunk q ^ ((l >> 1) & 3)
+                    const uint32_t pos = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+                    *reinterpret_cast<uint4*>(blk + pos) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                if (col0 + 32 <= args.N) {
-                    uint4* dst = reinterpret_cast<uint4*>(drow + col0);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                } else {
-                    const uint16_t* p16 = reinterpret_cast<const uint16_t*>(packed);
-                    uint16_t* d16 = reinterpret_cast<uint16_t*>(drow);
-                    for (int j = 0; j < 32 && col0 + j < args.N; ++j) d16[col0 + j] = p16[j];
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && m0 + (int)quarter * 32 < args.M && n0 + c * 32 < args.N) {
+                    tma_store_2d(&tm_d, blk, n0 + c * 32, m0 + (int)quarter * 32);
+                    bulk_commit_group();
                 }
             }
         }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();
-    __syncthreads();
+    if constexpr (C::PAIR)
+        cluster_sync();  // the leader's MMAs into the peer's TMEM are done before either frees it
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if constexpr (C::PAIR)
+            tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else
+            tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 

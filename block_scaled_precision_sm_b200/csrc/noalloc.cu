@@ -21,7 +21,8 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB
 
-// Packed SFA words at offset 0, packed SFB words at the next 256-byte boundary.
+// Packed SFA words at offset 0, packed SFB words and then the GEMM's scale chunks at the
+// next 256-byte boundaries.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDev = 64;
@@ -63,10 +64,13 @@ extern "C" int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const vo
     const int mn_b = (N + sfb_gran_n - 1) / sfb_gran_n;
     if (lda < K || ldb < K || ldd < N || ld_sfa_in < kb || ld_sfb_in < kb) return BSP_ERR_SHAPE;
     if (lda % 16 || ldb % 16 || (ldd * 2) % 16) return BSP_ERR_ALIGN;
-    // scratch: packed words for M and for ceil(N/g) scale rows, leading dimensions rounded to 8
+    // scratch: packed words for M and for ceil(N/g) scale rows (leading dimensions rounded to 8),
+    // then the tensor-core layout of those words that the GEMM loads
     const int64_t ld_a = round_up(M, 8), ld_b = round_up(mn_b, 8);
     const int64_t off_b = round_up((int64_t)words * ld_a * 2, 256);
-    if (off_b + (int64_t)words * ld_b * 2 > (int64_t)kScratchBytes) return BSP_ERR_UNSUPPORTED;
+    const int64_t off_chunks = round_up(off_b + (int64_t)words * ld_b * 2, 256);
+    const int64_t chunk_bytes = bsp::detail::gemm_fp8_scale_scratch_bytes(M, N, K, sfb_gran_n);
+    if (off_chunks + chunk_bytes > (int64_t)kScratchBytes) return BSP_ERR_UNSUPPORTED;
     void* scratch = nullptr;
     if (const int rc = scratch_address(&scratch)) return rc;
     unsigned char* sfa_w = static_cast<unsigned char*>(scratch);
@@ -79,5 +83,5 @@ extern "C" int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const vo
     if (const int rc = bsp::detail::launch_sf_transform_u8(sfb_e8m0, mn_b, kb, ld_sfb_in, sfb_w, ld_b, status, st))
         return rc;
     return bsp::detail::launch_gemm_fp8_packed(A, sfa_w, B, sfb_w, D, M, N, K, lda, ldb, ldd, ld_a, ld_b,
-                                               sfb_gran_n, status, st);
+                                               sfb_gran_n, status, sfa_w + off_chunks, st);
 }
