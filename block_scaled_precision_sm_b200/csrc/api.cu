@@ -153,14 +153,14 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? BSP_OK : BSP_ERR_CUDA;
 }
 
-//                       kind        BN   stages sf_stages grouped pair
-using CfgBF16P = GemmCfg<Kind::BF16, 224, 6, 1, false, true>;
-using CfgFP8P = GemmCfg<Kind::FP8, 224, 6, 3, false, true>;
-using CfgFP4P = GemmCfg<Kind::FP4, 224, 6, 6, false, true>;
-using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, 1, false, false>;
-using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, 2, false, false>;
-using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, 4, false, false>;
-using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, 2, true, false>;
+//                       kind        BN   stages grouped pair
+using CfgBF16P = GemmCfg<Kind::BF16, 224, 6, false, true>;
+using CfgFP8P = GemmCfg<Kind::FP8, 224, 6, false, true>;
+using CfgFP4P = GemmCfg<Kind::FP4, 224, 6, false, true>;
+using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
+using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
+using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
+using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 
 // Problem description shared by the GEMM entry points.
 struct Operands {

@@ -6,13 +6,13 @@
 // signals, "DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Reúso de
 // operandos e pipelining na prática", rebuilt for Blackwell):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) into an S-stage shared-memory
-//               ring ("full"/"empty" mbarriers, transaction-counted), and every SF_PERIOD K
-//               steps one chunk of scale words per operand into a small ring ("sf_full" /
-//               "sf_empty").  The chunks were laid out beforehand (sf_layout.cuh) exactly as
-//               the scale copy reads them, so no thread rearranges scales on chip.
-//   warp 1      owns TMEM; in the MMA-issuing CTA one elected lane issues tcgen05.cp of each
-//               scale chunk into a rotating TMEM slot and the tcgen05.mma instructions,
-//               committing to the "empty" / "sf_empty" barriers.
+//               ring ("full"/"empty" mbarriers, transaction-counted); the first stage of every
+//               scale group (SF_PERIOD K steps) also carries one chunk of scale words per
+//               operand, laid out beforehand (sf_layout.cuh) exactly as the scale copy reads
+//               them, so no thread rearranges scales on chip.
+//   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers and
+//               issues tcgen05.cp of each scale chunk into a rotating TMEM slot and the
+//               tcgen05.mma instructions, committing each stage to its "empty" barrier.
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in TMEM so the
 //               next tile's MMAs overlap), round to bf16, stage 32 x 32 blocks in a swizzled
 //               shared-memory buffer (two per warp) and TMA-store them to D.
@@ -62,7 +62,7 @@ struct GemmArgs {
     unsigned long long timeout_ns;
 };
 
-template <Kind KIND, int BLOCK_N_, int STAGES_, int SF_STAGES_, bool GROUPED_, bool PAIR_>
+template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
     static constexpr bool PAIR = PAIR_;
@@ -72,7 +72,6 @@ struct GemmCfg {
     static constexpr int BN = BLOCK_N_;         // columns per tile
     static constexpr int BN_CTA = BN / CTAS;    // B rows loaded per CTA
     static constexpr int STAGES = STAGES_;
-    static constexpr int SF_STAGES = SF_STAGES_;
     static constexpr bool GROUPED = GROUPED_;
     static constexpr bool SCALED = KIND != Kind::BF16;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && BN_CTA % 8 == 0, "BLOCK_N");
@@ -104,12 +103,12 @@ struct GemmCfg {
     // Shared memory map (offsets from a 1024-byte aligned base).
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;  // a scale chunk buffer per stage
     // epilogue staging: per epilogue warp two 32 x 32 bf16 blocks (64-byte swizzle)
     static constexpr int EPI_BLOCK = 32 * 32 * 2;
-    static constexpr int OFF_EPI = ((OFF_SF + (SCALED ? SF_STAGES * SF_STAGE_BYTES : 0) + 1023) / 1024) * 1024;
-    // full, empty [STAGES]; sf_full, sf_empty [SF_STAGES]; tmem_full, tmem_empty [2]; drain
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_STAGES + 5;
+    static constexpr int OFF_EPI = ((OFF_SF + STAGES * SF_STAGE_BYTES + 1023) / 1024) * 1024;
+    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain
+    static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
@@ -190,9 +189,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bars;
     uint64_t* empty = full + C::STAGES;
-    uint64_t* sf_full = empty + C::STAGES;
-    uint64_t* sf_empty = sf_full + C::SF_STAGES;
-    uint64_t* tmem_full = sf_empty + C::SF_STAGES;
+    uint64_t* tmem_full = empty + C::STAGES;
     uint64_t* tmem_empty = tmem_full + 2;
     uint64_t* drain = tmem_empty + 2;
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -210,10 +207,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-        }
-        for (int j = 0; j < C::SF_STAGES; ++j) {
-            mbar_init(&sf_full[j], 1);
-            mbar_init(&sf_empty[j], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full[b], 1);
@@ -252,7 +245,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t it = 0, git = 0;
+            uint32_t it = 0;
             bool ok = true;
             for (int t = worker; t < args.num_tiles && ok; t += workers) {
                 const Tile tl = tile_of(args, t);
@@ -268,52 +261,44 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
                 for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
-                    if constexpr (C::SCALED) {
-                        if (kb % C::SF_PERIOD == 0) {
-                            const uint32_t j = git % C::SF_STAGES, jph = (git / C::SF_STAGES) & 1u;
-                            if (!bounded_wait(&sf_empty[j], jph ^ 1u, args, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            if (leader) mbar_arrive_expect_tx(&sf_full[j], C::CTAS * C::SF_STAGE_BYTES);
-                            uint8_t* sf = smem + C::OFF_SF + j * C::SF_STAGE_BYTES;
-                            const int q = kb / C::SF_PERIOD;
-                            // chunk coordinates: (0, row tile, group [, expert])
-                            if constexpr (C::PAIR) {
-                                const uint32_t lead_sf = mapa_shared(smem_u32(&sf_full[j]), 0);
-                                tma_load_3d_pair(sf, &tm_sfa, lead_sf, 0, m0 / C::BM, q);
-                                tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_sf, 0, tl.n_blk, q);
-                            } else {
-                                tma_load_3d(sf, &tm_sfa, &sf_full[j], 0, m0 / C::BM, q);
-                                if constexpr (C::GROUPED)
-                                    tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &sf_full[j], 0, tl.n_blk, q, g);
-                                else
-                                    tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &sf_full[j], 0, tl.n_blk, q);
-                            }
-                            ++git;
-                        }
-                    }
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!bounded_wait(&empty[s], ph ^ 1u, args, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full[s], C::CTAS * (C::A_BYTES + C::B_BYTES));
+                    const bool sf_here = C::SCALED && kb % C::SF_PERIOD == 0;
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[s], C::CTAS * (C::A_BYTES + C::B_BYTES +
+                                                                   (sf_here ? C::SF_STAGE_BYTES : 0)));
                     uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
                     uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+                    uint8_t* sf = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
+                    const int q = kb / C::SF_PERIOD;
                     if constexpr (C::PAIR) {
                         const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), 0);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
                         tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
+                        if (sf_here) {
+                            // scale chunks: this CTA's A rows, all BN B rows of the tile
+                            tma_load_3d_pair(sf, &tm_sfa, lead_full, 0, m0 / C::BM, q);
+                            tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, tl.n_blk, q);
+                        }
                     } else {
                         tma_load_2d(sa, &tm_a, &full[s], kx, m0);
                         if constexpr (C::GROUPED)
                             tma_load_3d(sb, &tm_b, &full[s], kx, nb0, g);
                         else
                             tma_load_2d(sb, &tm_b, &full[s], kx, nb0);
+                        if (sf_here) {
+                            tma_load_3d(sf, &tm_sfa, &full[s], 0, m0 / C::BM, q);
+                            if constexpr (C::GROUPED)
+                                tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, tl.n_blk, q, g);
+                            else
+                                tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, tl.n_blk, q);
+                        }
                     }
                 }
             }
@@ -322,41 +307,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint32_t last = it < (uint32_t)C::STAGES ? it : (uint32_t)C::STAGES;
                 for (uint32_t j = it - last; j < it; ++j)
                     drain_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, args);
-                const uint32_t slast = git < (uint32_t)C::SF_STAGES ? git : (uint32_t)C::SF_STAGES;
-                for (uint32_t j = git - slast; j < git; ++j)
-                    drain_wait(&sf_full[j % C::SF_STAGES], (j / C::SF_STAGES) & 1u, args);
             }
         }
         __syncwarp();
     } else if (warp == 1 && leader) {
-        // ------------------------------------------------------------ MMA issue
-        uint32_t it = 0, lt = 0, git = 0;
-        bool ok = true;
-        for (int t = worker; t < args.num_tiles && ok; t += workers, ++lt) {
-            const uint32_t buf = lt & 1u;
-            const uint32_t aph = (lt >> 1) & 1u;
-            if (!warp_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + buf * C::BN;
-            uint32_t slot = 0;
-            for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
-                if constexpr (C::SCALED) {
-                    if (kb % C::SF_PERIOD == 0) {
-                        // copy this group's scale chunks into TMEM slot git % SF_SLOTS
-                        const uint32_t j = git % C::SF_STAGES, jph = (git / C::SF_STAGES) & 1u;
-                        if (!warp_wait(&sf_full[j], jph, args, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        slot = git % C::SF_SLOTS;
-                        if (lane == 0) {
+        // ------------------------------------------------------------ MMA issue (one lane)
+        if (lane == 0) {
+            uint32_t it = 0, lt = 0, git = 0;
+            bool ok = true;
+            for (int t = worker; t < args.num_tiles && ok; t += workers, ++lt) {
+                const uint32_t buf = lt & 1u;
+                const uint32_t aph = (lt >> 1) & 1u;
+                if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * C::BN;
+                uint32_t slot = 0;
+                for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!bounded_wait(&full[s], ph, args, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if constexpr (C::SCALED) {
+                        if (kb % C::SF_PERIOD == 0) {
+                            // copy this group's scale chunks (carried by this stage) into TMEM slot
+                            // git % SF_SLOTS; copies and MMAs run in issue order on the tensor pipe
+                            slot = git % C::SF_SLOTS;
+                            ++git;
                             const uint32_t sfa_col = C::ACC_COLS + slot * C::SF_SLOT_COLS;
                             const uint32_t sfb_col = sfa_col + C::SFA_COLS;
-                            const uint8_t* ua = smem + C::OFF_SF + j * C::SF_STAGE_BYTES;
+                            const uint8_t* ua = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
                             const uint8_t* ub = ua + C::SFA_CHUNK;
 #pragma unroll
                             for (int u = 0; u < C::UT_WORDS; ++u) {
@@ -375,24 +360,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                         tc_cp_32x128b_warpx4(col, d);
                                 }
                             }
-                            // the chunk buffers are free once these copies completed
-                            if constexpr (C::PAIR)
-                                tc_commit_pair_mc(&sf_empty[j], kPairMask);
-                            else
-                                tc_commit(&sf_empty[j]);
                         }
-                        __syncwarp();
-                        ++git;
                     }
-                }
-                const int s = it % C::STAGES;
-                const uint32_t ph = (it / C::STAGES) & 1u;
-                if (!warp_wait(&full[s], ph, args, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
                     const uint64_t adesc = smem_desc_k_sw128(smem + C::OFF_A + s * C::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + s * C::B_BYTES);
                     const uint32_t sfa_t = tmem_base + C::ACC_COLS + slot * C::SF_SLOT_COLS;
@@ -425,24 +394,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                 tc_mma_mxf4(d_tmem, ad, bd, id, sfa_t + 4 * u, sfb_t + 4 * C::SFB_ATOMS * u, acc);
                         }
                     }
+                    // the stage (A, B and any scale chunk) is free once these MMAs and copies completed
                     if constexpr (C::PAIR)
                         tc_commit_pair_mc(&empty[s], kPairMask);
                     else
                         tc_commit(&empty[s]);
                 }
-                __syncwarp();
-            }
-            if (!ok) break;
-            if (lane == 0) {
+                if (!ok) break;
                 if constexpr (C::PAIR)
                     tc_commit_pair_mc(&tmem_full[buf], kPairMask);
                 else
                     tc_commit(&tmem_full[buf]);
             }
-            __syncwarp();
-        }
-        // Wind down: every MMA and scale copy this warp issued has completed.
-        if (lane == 0) {
+            // Wind down: every MMA and scale copy this lane issued has completed.
             if constexpr (C::PAIR)
                 tc_commit_pair(drain);
             else
