@@ -45,6 +45,7 @@ PAGES_BF16_TFLOPS = 431.0
 NOMINAL_RATIO = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}  # dense tensor peak relative to bf16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["block_scaled_precision_sm_b200/csrc/gemm.cuh", "block_scaled_precision_sm_b200/csrc/ptx.cuh",
+                  "block_scaled_precision_sm_b200/csrc/sf_layout.cuh", "block_scaled_precision_sm_b200/csrc/sf_transform.cuh",
                   "block_scaled_precision_sm_b200/csrc/api.cu"]
 
 
@@ -351,7 +352,8 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
             ev[1].record()
 
     ms = float(timer.run(f_fp4, args.warmup, reps)[:, 0].mean())
-    k, v = _gemm_entry("fp4_4096x7168x16384", gemm_flops(M, N, K), ms, bf16_peak * NOMINAL_RATIO["fp4"])
+    k, v = _gemm_entry("fp4_4096x7168x16384", gemm_flops(M, N, K), ms, bf16_peak * NOMINAL_RATIO["fp4"],
+                       {"traffic": profiled_traffic("gemm_fp4_4096x7168x16384.md")})
     out[k] = v
     del d4, sa, sb
 
@@ -398,7 +400,8 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
     fl_padded = gemm_flops(g["M"], 4096, 7168)
     k, v = _gemm_entry("grouped_fp8_32x32768x4096x7168", fl_valid, ms, bf16_peak * 2,
                        {"m_total_padded": int(g["M"]),
-                        "tflops_incl_padding": round(fl_padded / (ms * 1e-3) / 1e12, 1)})
+                        "tflops_incl_padding": round(fl_padded / (ms * 1e-3) / 1e12, 1),
+                        "traffic": profiled_traffic("gemm_grouped_fp8_32x32768x4096x7168.md")})
     out[k] = v
 
     # scale transform alone: config-3 SFA (fp32 scales [M_total, 56]) -> int16 words
@@ -417,7 +420,8 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
     moved = s32.numel() * 4 + w.numel() * 2
     out["sf_transform_fp32_36864x56"] = {"gbs": round(moved / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 5),
                                          "bytes": int(moved), "hbm_peak_gbs": peaks["hbm_gbs"],
-                                         "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+                                         "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                         "traffic": profiled_traffic("sf_transform_fp32_36864x56.md")}
     return out
 
 

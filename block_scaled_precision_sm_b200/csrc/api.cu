@@ -161,6 +161,19 @@ using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
 using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
 using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
+// M <= 128 with few 224-wide tiles: 64-wide tiles put ~3.5x more SMs on the (B-bandwidth-bound)
+// problem, and their 24 KB stages allow a deeper ring.
+using CfgBF16N = GemmCfg<Kind::BF16, 64, 8, false, false>;
+using CfgFP8N = GemmCfg<Kind::FP8, 64, 8, false, false>;
+using CfgFP4N = GemmCfg<Kind::FP4, 64, 8, false, false>;
+
+// Tile shape by problem shape: CTA pairs for M > 128; for M <= 128 single CTAs, 64 wide when
+// 224-wide tiles would leave most SMs idle.
+enum class Shape { Pair, Wide, Narrow };
+Shape pick_shape(int M, int N, int sms) {
+    if (M > 128) return Shape::Pair;
+    return (N + 223) / 224 * 2 <= sms ? Shape::Narrow : Shape::Wide;
+}
 
 // Problem description shared by the GEMM entry points.
 struct Operands {
@@ -318,7 +331,13 @@ int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
     const Operands o{nullptr, nullptr, nullptr, nullptr, 0, 0, 0, 0, (N + sfb_gran_n - 1) / sfb_gran_n, words};
     GemmArgs a{};
     a.M = M, a.N = N, a.K = K, a.sfb_gran = sfb_gran_n;
-    return M > 128 ? ScaleChunks<CfgFP8P>(o, a).bytes() : ScaleChunks<CfgFP8>(o, a).bytes();
+    int sms = 0;
+    if (device_facts_noalloc(&sms) != BSP_OK) sms = 148;
+    switch (pick_shape(M, N, sms)) {
+        case Shape::Pair: return ScaleChunks<CfgFP8P>(o, a).bytes();
+        case Shape::Wide: return ScaleChunks<CfgFP8>(o, a).bytes();
+        default: return ScaleChunks<CfgFP8N>(o, a).bytes();
+    }
 }
 
 int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
@@ -335,8 +354,11 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
     a.M = M, a.N = N, a.K = K;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    return M > 128 ? launch_gemm<CfgFP8P>(o, a, ctx, stream, scale_scratch)
-                   : launch_gemm<CfgFP8>(o, a, ctx, stream, scale_scratch);
+    switch (pick_shape(M, N, ctx.sms)) {
+        case Shape::Pair: return launch_gemm<CfgFP8P>(o, a, ctx, stream, scale_scratch);
+        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, ctx, stream, scale_scratch);
+        default: return launch_gemm<CfgFP8N>(o, a, ctx, stream, scale_scratch);
+    }
 }
 
 }  // namespace detail
@@ -362,7 +384,11 @@ int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K, int
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return M > 128 ? launch_gemm<CfgBF16P>(o, a, *ctx, st) : launch_gemm<CfgBF16>(o, a, *ctx, st);
+    switch (pick_shape(M, N, ctx->sms)) {
+        case Shape::Pair: return launch_gemm<CfgBF16P>(o, a, *ctx, st);
+        case Shape::Wide: return launch_gemm<CfgBF16>(o, a, *ctx, st);
+        default: return launch_gemm<CfgBF16N>(o, a, *ctx, st);
+    }
 }
 
 int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N, int K,
@@ -387,7 +413,11 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return M > 128 ? launch_gemm<CfgFP8P>(o, a, *ctx, st) : launch_gemm<CfgFP8>(o, a, *ctx, st);
+    switch (pick_shape(M, N, ctx->sms)) {
+        case Shape::Pair: return launch_gemm<CfgFP8P>(o, a, *ctx, st);
+        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, *ctx, st);
+        default: return launch_gemm<CfgFP8N>(o, a, *ctx, st);
+    }
 }
 
 int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N, int K,
@@ -409,7 +439,11 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return M > 128 ? launch_gemm<CfgFP4P>(o, a, *ctx, st) : launch_gemm<CfgFP4>(o, a, *ctx, st);
+    switch (pick_shape(M, N, ctx->sms)) {
+        case Shape::Pair: return launch_gemm<CfgFP4P>(o, a, *ctx, st);
+        case Shape::Wide: return launch_gemm<CfgFP4>(o, a, *ctx, st);
+        default: return launch_gemm<CfgFP4N>(o, a, *ctx, st);
+    }
 }
 
 int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void* B, const void* sfb, void* D,

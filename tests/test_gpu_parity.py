@@ -247,3 +247,25 @@ def test_wait_timeout_is_reported_and_context_survives(ops, orc):
     D = ops.gemm_fp8_nt(*args)
     _status_ok(ops)
     check_gemm(bf16_to_f64(D), orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"]), "after timeout")
+
+
+# ------------------------------------------------------------------ tile shapes
+
+@pytest.mark.parametrize("kind", ["fp8", "bf16", "fp4"])
+def test_wide_single_cta_tiles(ops, orc, kind):
+    # M <= 128 with more than 74 tiles of 224 columns: single-CTA 224-wide tiles
+    m, n, k = 96, 16640, 256
+    if kind == "fp8":
+        p = inputs.dense_fp8_problem(m, n, k, seed=77)
+        D = ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]))
+        ref = orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"])
+    elif kind == "bf16":
+        p = inputs.dense_bf16_problem(m, n, k, seed=78)
+        D = ops.gemm_bf16_nt(to_dev(p["A"], torch.bfloat16), to_dev(p["B"], torch.bfloat16))
+        ref = orc.gemm_bf16(p["A"], p["B"])
+    else:
+        p = inputs.dense_fp4_problem(m, n, k, seed=79)
+        D = ops.gemm_fp4_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]))
+        ref = orc.gemm_fp4(p["A"], p["sfa"], p["B"], p["sfb"])
+    _status_ok(ops)
+    check_gemm(bf16_to_f64(D), ref, f"{kind} wide single-CTA")
