@@ -65,6 +65,31 @@ def parse():
     return ap.parse_args()
 
 
+def rank_env():
+    """(rank, world size, local rank) of this process, as torchrun sets them."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -181,25 +206,12 @@ def run_ours(args):
 
     from block_scaled_precision_sm_b200 import ops
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     peaks, peak_kind = load_peaks()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     timer = Timer(torch)
     kb = K // 128
@@ -225,7 +237,7 @@ def run_ours(args):
         timer.flush.zero_()
         step(None)
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
@@ -236,13 +248,13 @@ def run_ours(args):
     launches = ops.kernel_launches() - launches0
     clocks = sampler.stop()
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     status = ops.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    step_ms = max_over_ranks(float(spans.sum(axis=1).mean()))
-    gemm_ms = max_over_ranks(float(spans[:, 1].mean()))
+    step_ms = max_over_ranks(float(spans.sum(axis=1).mean()), world, "cuda")
+    gemm_ms = max_over_ranks(float(spans[:, 1].mean()), world, "cuda")
     flops = gemm_flops(M, N, K)
     value = world * flops / (step_ms * 1e-3) / 1e12
     fp8_peak = peaks["bf16_tflops"] * NOMINAL_RATIO["fp8"]
@@ -287,7 +299,7 @@ def run_ours(args):
             ev[1].record()
 
     e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms = max_over_ranks(float(timer.run(e2e_step, 2, e2e_steps)[:, 0].mean()))
+    e2e_ms = max_over_ranks(float(timer.run(e2e_step, 2, e2e_steps)[:, 0].mean()), world, "cuda")
     line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
                    "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                    "api": "ops.gemm_fp8_nt with uint8 UE8M0 scales (packed inside the call)"}
@@ -447,10 +459,9 @@ def cpu_baseline(p, budget_s: float = 10.0):
 # ---------------------------------------------------------------- reference arm (the oracle)
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank, world, _ = rank_env()
     if rank != 0:
-        return
+        return  # the CPU reference runs once, on rank 0
     import oracle
 
     oracle.build()

@@ -149,9 +149,10 @@ int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t l
  *   status    device int, output: set to 0 by the call, then latched by its kernels like the
  *             status word of the other calls (BSP_ERR_TIMEOUT, BSP_ERR_DEVICE_CHECK); read it
  *             after the stream has finished.
- * Limit: the packed words, round_up(M,8) + round_up(ceil(N/g),8) int16 per K pair (the SFA
- * part rounded up to 256 bytes), must fit in 4 MiB — for example M up to about 32000 at
- * K = 16384; larger calls return BSP_ERR_UNSUPPORTED and launch nothing.
+ * Limit: the packed words (round_up(M,8) + round_up(ceil(N/g),8) int16 per K pair) plus the
+ * tensor-core layout of them the GEMM loads (one 32-bit word per row and four K blocks, B
+ * rows counted per 224-row tile) must fit in 4 MiB — for example M up to about 12000 at
+ * N = 7168, K = 16384; larger calls return BSP_ERR_UNSUPPORTED and launch nothing.
  * Every call shares the one scratch array and overwrites it: calls that overlap on the GPU
  * (different streams, or different host threads on one device) race on it and must be
  * ordered by the caller.  The first call on each device looks up the array's device address

@@ -86,3 +86,15 @@ def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(ImportError):
         _lib.load()
+
+
+def test_noalloc_scratch_limit_without_gpu(lib):
+    # the size check comes before any CUDA call: 13000 rows of A scales at K = 16384 do not fit
+    vp = ctypes.c_void_p
+    good = vp(0x10000)
+    st = vp(0x10004)
+    assert lib.gemm_fp8_nt_noalloc(good, good, good, good, good, st, 13000, 7168, 16384, 16384, 16384, 7168,
+                                   128, 128, 128, None) == -4
+    # 12000 rows fit: the call gets past the size check (and then fails without a GPU)
+    assert lib.gemm_fp8_nt_noalloc(good, good, good, good, good, st, 12000, 7168, 16384, 16384, 16384, 7168,
+                                   128, 128, 128, None) != -4
