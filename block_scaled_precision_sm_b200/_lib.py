@@ -22,6 +22,7 @@ SIGNATURES = {
     "bsp_status_string": (ctypes.c_char_p, [_i]),
     "bsp_set_wait_timeout_ns": (_u64, [_u64]),
     "bsp_kernel_launches": (_u64, []),
+    "bsp_gemm_plan": (_i, [_i, _i, _i, _i, _vp]),
 }
 
 STATUS = {0: "BSP_OK", -1: "BSP_ERR_ARG", -2: "BSP_ERR_ALIGN", -3: "BSP_ERR_SHAPE", -4: "BSP_ERR_UNSUPPORTED",

@@ -74,6 +74,8 @@ int ensure_ctx(DeviceCtx** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int64_t round_up_i(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
 // Encode a tiled tensor map; dims/box are innermost first, strides (bytes) for dims 1..rank-1.
 int encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
            const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
@@ -103,22 +105,104 @@ int operand_map_3d(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t 
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Co-resident workers (CTAs or CTA pairs) of config C on the current device: a persistent
+// grid larger than this would serialise its last workers.
+template <class C>
+int max_workers_of(const DeviceCtx& ctx, int* out) {
+    static std::once_flag once[kMaxDevices];
+    static int workers[kMaxDevices];
+    static cudaError_t err[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSP_ERR_CUDA;
+    std::call_once(once[dev], [&] {
+        err[dev] = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C::CTAS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(C::CTAS * (ctx.sms / C::CTAS));
+        int clusters = 0;
+        if (err[dev] == cudaSuccess) err[dev] = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<C>, &cfg);
+        workers[dev] = clusters > 0 ? clusters : ctx.sms / C::CTAS;
+    });
+    if (err[dev] != cudaSuccess) return BSP_ERR_CUDA;
+    *out = workers[dev];
+    return BSP_OK;
+}
+
+// Tail plan: how many whole tiles, and into how many K slices the rest is cut.  The tiles
+// left over after the last full wave of workers are split when at least two slices of
+// eight or more K steps fit per tile, up to 16 slices, so that the last wave keeps most
+// workers busy instead of a few.
+struct TailPlan {
+    int tiles, full_tiles, splits, tail_tiles, num_work;
+};
+
+TailPlan plan_tail(int tiles, int num_kb, int period, int workers, bool allow) {
+    TailPlan p{tiles, tiles, 1, 0, tiles};
+    const int rem = tiles % workers;
+    if (!allow || rem == 0) return p;
+    const int groups = (num_kb + period - 1) / period;
+    int s = workers / rem;
+    s = s < 16 ? s : 16;
+    s = s < groups ? s : groups;
+    while (s >= 2 && num_kb / s < 8) --s;
+    if (s < 2) return p;
+    p.full_tiles = tiles - rem;
+    p.splits = s;
+    p.tail_tiles = rem;
+    p.num_work = p.full_tiles + rem * s;
+    return p;
+}
+
+template <class C>
+int64_t tail_ws_bytes(const TailPlan& p) {
+    return p.splits > 1 ? (int64_t)p.tail_tiles * p.splits * C::TILE_M * C::BN * 4 : 0;
+}
+template <class C>
+int64_t tail_count_bytes(const TailPlan& p) {
+    return p.splits > 1 ? round_up_i((int64_t)p.tail_tiles * C::CTAS * 4 * 4, 256) : 0;
+}
+
+// Launch config C with the split-tail plan `p` (ws: its workspace, count: its zeroed counters).
 template <class C>
 int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
-           GemmArgs a, const DeviceCtx& ctx, cudaStream_t stream) {
+           GemmArgs a, const TailPlan& p, float* ws, int* count, const DeviceCtx& ctx, cudaStream_t stream) {
     // D: bf16 [M][ldd], stored in 32 x 32 blocks through a 64-byte-swizzled staging buffer
-    CUtensorMap td;
+    CUtensorMap td, tw;
     {
         const cuuint64_t dims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
         const cuuint64_t strides[1] = {(cuuint64_t)(a.ldd * 2)};
         const cuuint32_t box[2] = {32, 32};
         BSP_TRY(encode(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.D, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B));
     }
-    static std::once_flag attr_once[kMaxDevices];
-    static int max_workers[kMaxDevices];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaError_t attr_err = cudaSuccess;
+    if (p.splits > 1) {
+        // workspace: fp32 [split tiles * splits * TILE_M][BN], stored in 32 x 32 blocks
+        const cuuint64_t dims[2] = {(cuuint64_t)C::BN, (cuuint64_t)p.tail_tiles * p.splits * C::TILE_M};
+        const cuuint64_t strides[1] = {(cuuint64_t)C::BN * 4};
+        const cuuint32_t box[2] = {32, 32};
+        BSP_TRY(encode(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ws, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        tw = td;  // not read
+    }
+    int max_workers = 0;
+    BSP_TRY(max_workers_of<C>(ctx, &max_workers));
+    a.num_tiles = p.tiles;
+    a.full_tiles = p.full_tiles;
+    a.splits = p.splits;
+    a.num_work = p.num_work;
+    a.ws = ws;
+    a.tail_count = count;
+    a.group_m = 16;
+    a.status = ctx.status;
+    a.timeout_ns = g_timeout_ns.load();
+    const int workers = a.num_work < max_workers ? a.num_work : max_workers;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -130,33 +214,22 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    std::call_once(attr_once[dev], [&] {
-        attr_err = cudaFuncSetAttribute(gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        int clusters = 0;
-        cfg.gridDim = dim3(C::CTAS * (ctx.sms / C::CTAS));
-        if (attr_err == cudaSuccess)
-            attr_err = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<C>, &cfg);
-        // a persistent grid larger than what is co-resident would serialise its last workers
-        max_workers[dev] = clusters > 0 ? clusters : ctx.sms / C::CTAS;
-    });
-    if (attr_err != cudaSuccess) return BSP_ERR_CUDA;
-    a.m_blocks = (a.M + C::TILE_M - 1) / C::TILE_M;
-    a.n_blocks = (a.N + C::BN - 1) / C::BN;
-    a.num_tiles = a.m_blocks * a.n_blocks;
-    a.group_m = 16;
-    a.status = ctx.status;
-    a.timeout_ns = g_timeout_ns.load();
-    const int workers = a.num_tiles < max_workers[dev] ? a.num_tiles : max_workers[dev];
     cfg.gridDim = dim3(C::CTAS * workers);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, td, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, td, tw, a);
     g_launches.fetch_add(1);
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? BSP_OK : BSP_ERR_CUDA;
 }
 
-//                       kind        BN   stages grouped pair
-using CfgBF16P = GemmCfg<Kind::BF16, 224, 6, false, true>;
-using CfgFP8P = GemmCfg<Kind::FP8, 224, 6, false, true>;
-using CfgFP4P = GemmCfg<Kind::FP4, 224, 6, false, true>;
+//                          kind        BN   stages grouped pair  accumulators
+using CfgBF16P224 = GemmCfg<Kind::BF16, 224, 6, false, true>;
+using CfgFP8P224 = GemmCfg<Kind::FP8, 224, 6, false, true>;
+using CfgFP4P224 = GemmCfg<Kind::FP4, 224, 6, false, true>;
+// 256 x 256 pair tiles keep the tensor pipe busier than 256 x 224 ones (measured: about 8%
+// more throughput per tile), but two 256-column accumulators leave no TMEM for the scales,
+// so these run with one accumulator and an epilogue that empties it into registers at once.
+using CfgBF16P256 = GemmCfg<Kind::BF16, 256, 6, false, true, 1>;
+using CfgFP8P256 = GemmCfg<Kind::FP8, 256, 6, false, true, 1>;
+using CfgFP4P256 = GemmCfg<Kind::FP4, 256, 5, false, true, 1>;
 using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
 using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
@@ -167,11 +240,29 @@ using CfgBF16N = GemmCfg<Kind::BF16, 64, 8, false, false>;
 using CfgFP8N = GemmCfg<Kind::FP8, 64, 8, false, false>;
 using CfgFP4N = GemmCfg<Kind::FP4, 64, 8, false, false>;
 
-// Tile shape by problem shape: CTA pairs for M > 128; for M <= 128 single CTAs, 64 wide when
-// 224-wide tiles would leave most SMs idle.
-enum class Shape { Pair, Wide, Narrow };
-Shape pick_shape(int M, int N, int sms) {
-    if (M > 128) return Shape::Pair;
+// Tile shape by problem shape.  M > 128: CTA pairs, 256 or 224 columns wide, whichever
+// finishes first by a model of the waves (tile time proportional to its MMA work, 224-wide
+// tiles 8% less efficient, a split tail paying for its longest slice plus about four K steps
+// of reduction).  M <= 128: single CTAs, 64 wide when 224-wide tiles would leave most SMs
+// idle.
+enum class Shape { Pair256, Pair224, Wide, Narrow };
+Shape pick_shape(int M, int N, int num_kb, int period, int sms) {
+    if (M > 128) {
+        const int workers = sms / 2;
+        const auto cost = [&](int bn, double eff) {
+            const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
+            const TailPlan p = plan_tail(tiles, num_kb, period, workers, true);
+            double steps;
+            if (p.splits > 1) {
+                const int groups = (num_kb + period - 1) / period;
+                steps = (double)(p.full_tiles / workers) * num_kb + (double)((groups + p.splits - 1) / p.splits) * period + 4.0;
+            } else {
+                steps = (double)((tiles + workers - 1) / workers) * num_kb;
+            }
+            return steps * 256.0 * bn / eff;
+        };
+        return cost(256, 1.0) <= cost(224, 0.92) ? Shape::Pair256 : Shape::Pair224;
+    }
     return (N + 223) / 224 * 2 <= sms ? Shape::Narrow : Shape::Wide;
 }
 
@@ -203,13 +294,14 @@ struct ScaleChunks {
     int64_t bytes() const { return a_bytes + b_bytes; }
 };
 
+// Scale chunks of both operands, and `zero_bytes` (a multiple of 16) zeroed at `zero`.
 int launch_sf_layout(const void* in_a, const SfLayout& pa, void* out_a, const void* in_b, const SfLayout& pb,
-                     void* out_b, cudaStream_t stream) {
-    const int64_t total = sf_layout_words(pa) + sf_layout_words(pb);
+                     void* out_b, void* zero, int64_t zero_bytes, cudaStream_t stream) {
+    const int64_t total = sf_layout_words(pa) + sf_layout_words(pb) + zero_bytes / 16;
     const int64_t blocks = (total + 255) / 256;
     sf_tmem_layout_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
         static_cast<const uint16_t*>(in_a), pa, static_cast<uint32_t*>(out_a), static_cast<const uint16_t*>(in_b),
-        pb, static_cast<uint32_t*>(out_b));
+        pb, static_cast<uint32_t*>(out_b), static_cast<uint4*>(zero), zero_bytes / 16);
     g_launches.fetch_add(1);
     return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
 }
@@ -251,10 +343,43 @@ int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int 
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Encode the tensor maps for config C and launch it.  Scaled kinds first lay the scales out
-// as TMEM chunks in `ws` (stream-ordered scratch on the caller's stream when ws is null).
+// Tiles, K steps and the tail plan of config C for this problem on this device.
 template <class C>
-int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_t stream, void* ws = nullptr) {
+int plan_gemm(GemmArgs& a, const DeviceCtx& ctx, TailPlan* p, int* workers) {
+    const int64_t row_bytes = C::kind == Kind::FP4 ? a.K / 2 : (C::kind == Kind::BF16 ? (int64_t)a.K * 2 : a.K);
+    a.num_kb = (int)((row_bytes + 127) / 128);
+    a.m_blocks = (a.M + C::TILE_M - 1) / C::TILE_M;
+    a.n_blocks = (a.N + C::BN - 1) / C::BN;
+    int max_workers = 0;
+    BSP_TRY(max_workers_of<C>(ctx, &max_workers));
+    *p = plan_tail(a.m_blocks * a.n_blocks, a.num_kb, C::SF_PERIOD, max_workers, !C::GROUPED);
+    *workers = max_workers;
+    return BSP_OK;
+}
+
+template <class C>
+int describe_plan(int M, int N, int K, const DeviceCtx& ctx, int32_t* out) {
+    GemmArgs a{};
+    a.M = M, a.N = N, a.K = K;
+    TailPlan p;
+    int max_workers = 0;
+    BSP_TRY(plan_gemm<C>(a, ctx, &p, &max_workers));
+    out[0] = C::TILE_M;
+    out[1] = C::BN;
+    out[2] = p.splits;
+    out[3] = p.tail_tiles;
+    out[4] = p.num_work;
+    out[5] = p.num_work < max_workers ? p.num_work : max_workers;
+    return BSP_OK;
+}
+
+// Encode the tensor maps for config C and launch it.  Scratch (stream-ordered, from the
+// caller's stream, unless `fixed` is given): the scale chunks of scaled kinds, then the
+// split tail's counters (zeroed by the scale layout pass, or a memset) and workspace.  With
+// `fixed` scratch of `fixed_bytes`, the tail is split only if its workspace fits.
+template <class C>
+int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_t stream, void* fixed = nullptr,
+                int64_t fixed_bytes = 0) {
     constexpr bool bf16 = C::kind == Kind::BF16;
     const auto dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const int es = bf16 ? 2 : 1;
@@ -265,25 +390,42 @@ int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_
         BSP_TRY(operand_map_3d(&tb, o.B, a.K, a.N, o.groups, C::BN_CTA));
     else
         BSP_TRY(operand_map(&tb, dt, es, o.B, row_elems, a.N, o.ldb, C::BN_CTA));
-    a.num_kb = (int)((row_elems * es + 127) / 128);
-    if constexpr (!C::SCALED) {
-        return launch<C>(ta, tb, ta, tb, a, ctx, stream);
-    } else {
+    TailPlan p;
+    int max_workers = 0;
+    BSP_TRY(plan_gemm<C>(a, ctx, &p, &max_workers));
+    int64_t chunk_bytes = 0;
+    SfLayout la{}, lb{};
+    if constexpr (C::SCALED) {
         const ScaleChunks<C> sc(o, a);
-        bool owned = false;
-        if (ws == nullptr) {
-            BSP_TRY(scratch_alloc(&ws, (size_t)sc.bytes(), stream));
-            owned = true;
-        }
-        char* wa = static_cast<char*>(ws);
-        char* wb = wa + sc.a_bytes;
-        int rc = launch_sf_layout(o.sfa, sc.a, wa, o.sfb, sc.b, wb, stream);
-        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, sc.a.tiles, sc.a.q, 1);
-        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, sc.b.tiles, sc.b.q, C::GROUPED ? -o.groups : 1);
-        if (rc == BSP_OK) rc = launch<C>(ta, tb, tsa, tsb, a, ctx, stream);
-        if (owned && cudaFreeAsync(ws, stream) != cudaSuccess && rc == BSP_OK) rc = BSP_ERR_CUDA;
-        return rc;
+        chunk_bytes = sc.bytes();
+        la = sc.a, lb = sc.b;
     }
+    int64_t tail_bytes = tail_count_bytes<C>(p) + tail_ws_bytes<C>(p);
+    if (fixed != nullptr && chunk_bytes + tail_bytes > fixed_bytes) {
+        p = plan_tail(p.tiles, a.num_kb, C::SF_PERIOD, max_workers, false);
+        tail_bytes = 0;
+    }
+    void* scratch = fixed;
+    const bool owned = fixed == nullptr && chunk_bytes + tail_bytes > 0;
+    if (owned) BSP_TRY(scratch_alloc(&scratch, (size_t)(chunk_bytes + tail_bytes), stream));
+    char* base = static_cast<char*>(scratch);
+    int* count = tail_bytes ? reinterpret_cast<int*>(base + chunk_bytes) : nullptr;
+    float* ws = tail_bytes ? reinterpret_cast<float*>(base + chunk_bytes + tail_count_bytes<C>(p)) : nullptr;
+    int rc = BSP_OK;
+    if constexpr (C::SCALED) {
+        char* wa = base;
+        char* wb = wa + ScaleChunks<C>(o, a).a_bytes;
+        rc = launch_sf_layout(o.sfa, la, wa, o.sfb, lb, wb, count, tail_bytes ? tail_count_bytes<C>(p) : 0, stream);
+        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1);
+        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1);
+    } else {
+        tsa = ta, tsb = tb;  // not read
+        if (tail_bytes && cudaMemsetAsync(count, 0, (size_t)tail_count_bytes<C>(p), stream) != cudaSuccess)
+            rc = BSP_ERR_CUDA;
+    }
+    if (rc == BSP_OK) rc = launch<C>(ta, tb, tsa, tsb, a, p, ws, count, ctx, stream);
+    if (owned && cudaFreeAsync(scratch, stream) != cudaSuccess && rc == BSP_OK) rc = BSP_ERR_CUDA;
+    return rc;
 }
 
 int check_ld(int64_t ld, int64_t min_elems, int esize) {
@@ -333,8 +475,9 @@ int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
     a.M = M, a.N = N, a.K = K, a.sfb_gran = sfb_gran_n;
     int sms = 0;
     if (device_facts_noalloc(&sms) != BSP_OK) sms = 148;
-    switch (pick_shape(M, N, sms)) {
-        case Shape::Pair: return ScaleChunks<CfgFP8P>(o, a).bytes();
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, sms)) {
+        case Shape::Pair256: return ScaleChunks<CfgFP8P256>(o, a).bytes();
+        case Shape::Pair224: return ScaleChunks<CfgFP8P224>(o, a).bytes();
         case Shape::Wide: return ScaleChunks<CfgFP8>(o, a).bytes();
         default: return ScaleChunks<CfgFP8N>(o, a).bytes();
     }
@@ -342,7 +485,7 @@ int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
 
 int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
                            int K, int64_t lda, int64_t ldb, int64_t ldd, int64_t ld_sfa, int64_t ld_sfb,
-                           int sfb_gran_n, int* status, void* scale_scratch, cudaStream_t stream) {
+                           int sfb_gran_n, int* status, void* scratch, int64_t scratch_bytes, cudaStream_t stream) {
     DeviceCtx ctx;
     BSP_TRY(device_facts_noalloc(&ctx.sms));
     ctx.ready = true;
@@ -354,10 +497,11 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
     a.M = M, a.N = N, a.K = K;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    switch (pick_shape(M, N, ctx.sms)) {
-        case Shape::Pair: return launch_gemm<CfgFP8P>(o, a, ctx, stream, scale_scratch);
-        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, ctx, stream, scale_scratch);
-        default: return launch_gemm<CfgFP8N>(o, a, ctx, stream, scale_scratch);
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx.sms)) {
+        case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, ctx, stream, scratch, scratch_bytes);
+        case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, ctx, stream, scratch, scratch_bytes);
+        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, ctx, stream, scratch, scratch_bytes);
+        default: return launch_gemm<CfgFP8N>(o, a, ctx, stream, scratch, scratch_bytes);
     }
 }
 
@@ -384,8 +528,9 @@ int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K, int
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (pick_shape(M, N, ctx->sms)) {
-        case Shape::Pair: return launch_gemm<CfgBF16P>(o, a, *ctx, st);
+    switch (pick_shape(M, N, (K + 63) / 64, CfgBF16::SF_PERIOD, ctx->sms)) {
+        case Shape::Pair256: return launch_gemm<CfgBF16P256>(o, a, *ctx, st);
+        case Shape::Pair224: return launch_gemm<CfgBF16P224>(o, a, *ctx, st);
         case Shape::Wide: return launch_gemm<CfgBF16>(o, a, *ctx, st);
         default: return launch_gemm<CfgBF16N>(o, a, *ctx, st);
     }
@@ -413,8 +558,9 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (pick_shape(M, N, ctx->sms)) {
-        case Shape::Pair: return launch_gemm<CfgFP8P>(o, a, *ctx, st);
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx->sms)) {
+        case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, *ctx, st);
+        case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, *ctx, st);
         case Shape::Wide: return launch_gemm<CfgFP8>(o, a, *ctx, st);
         default: return launch_gemm<CfgFP8N>(o, a, *ctx, st);
     }
@@ -439,8 +585,9 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = 1;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (pick_shape(M, N, ctx->sms)) {
-        case Shape::Pair: return launch_gemm<CfgFP4P>(o, a, *ctx, st);
+    switch (pick_shape(M, N, K / 256 + (K % 256 ? 1 : 0), CfgFP4::SF_PERIOD, ctx->sms)) {
+        case Shape::Pair256: return launch_gemm<CfgFP4P256>(o, a, *ctx, st);
+        case Shape::Pair224: return launch_gemm<CfgFP4P224>(o, a, *ctx, st);
         case Shape::Wide: return launch_gemm<CfgFP4>(o, a, *ctx, st);
         default: return launch_gemm<CfgFP4N>(o, a, *ctx, st);
     }
@@ -525,5 +672,35 @@ const char* bsp_status_string(int status) {
 uint64_t bsp_set_wait_timeout_ns(uint64_t ns) { return g_timeout_ns.exchange(ns); }
 
 uint64_t bsp_kernel_launches(void) { return g_launches.load(); }
+
+int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
+    if (!plan || M <= 0 || N <= 0 || K <= 0 || kind < 0 || kind > 3) return BSP_ERR_ARG;
+    DeviceCtx* ctx;
+    BSP_TRY(ensure_ctx(&ctx));
+    switch (kind) {
+        case 0:
+            switch (pick_shape(M, N, (K + 63) / 64, CfgBF16::SF_PERIOD, ctx->sms)) {
+                case Shape::Pair256: return describe_plan<CfgBF16P256>(M, N, K, *ctx, plan);
+                case Shape::Pair224: return describe_plan<CfgBF16P224>(M, N, K, *ctx, plan);
+                case Shape::Wide: return describe_plan<CfgBF16>(M, N, K, *ctx, plan);
+                default: return describe_plan<CfgBF16N>(M, N, K, *ctx, plan);
+            }
+        case 1:
+            switch (pick_shape(M, N, (K + 127) / 128, CfgFP8::SF_PERIOD, ctx->sms)) {
+                case Shape::Pair256: return describe_plan<CfgFP8P256>(M, N, K, *ctx, plan);
+                case Shape::Pair224: return describe_plan<CfgFP8P224>(M, N, K, *ctx, plan);
+                case Shape::Wide: return describe_plan<CfgFP8>(M, N, K, *ctx, plan);
+                default: return describe_plan<CfgFP8N>(M, N, K, *ctx, plan);
+            }
+        case 2:
+            switch (pick_shape(M, N, (K + 255) / 256, CfgFP4::SF_PERIOD, ctx->sms)) {
+                case Shape::Pair256: return describe_plan<CfgFP4P256>(M, N, K, *ctx, plan);
+                case Shape::Pair224: return describe_plan<CfgFP4P224>(M, N, K, *ctx, plan);
+                case Shape::Wide: return describe_plan<CfgFP4>(M, N, K, *ctx, plan);
+                default: return describe_plan<CfgFP4N>(M, N, K, *ctx, plan);
+            }
+        default: return describe_plan<CfgGrouped>(M, N, K, *ctx, plan);
+    }
+}
 
 }  // extern "C"

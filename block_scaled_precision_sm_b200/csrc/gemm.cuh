@@ -60,9 +60,21 @@ struct GemmArgs {
     int sfb_gran;              // 1 or 128 (FP8); 1 for FP4
     int* status;
     unsigned long long timeout_ns;
+    // Split tail: the first full_tiles tiles (in raster order) are computed whole, one per
+    // work item; each remaining tile is cut into `splits` slices along K.  Slice j stores its
+    // fp32 partial sums in its own workspace slot (ws: [split tiles][splits][TILE_M][BN]),
+    // counts itself in tail_count ([split tiles][CTAs][4 epilogue warps], zero on entry) and
+    // waits for the other slices; then slice j adds up all slots, in slot order, for its
+    // share of the rows and rounds them to bf16 in D.  The fixed order keeps the result
+    // identical from run to run.
+    int full_tiles;
+    int splits;
+    int num_work;  // full_tiles + (num_tiles - full_tiles) * splits
+    float* ws;
+    int* tail_count;
 };
 
-template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_>
+template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
     static constexpr bool PAIR = PAIR_;
@@ -74,6 +86,10 @@ struct GemmCfg {
     static constexpr int STAGES = STAGES_;
     static constexpr bool GROUPED = GROUPED_;
     static constexpr bool SCALED = KIND != Kind::BF16;
+    // TMEM accumulators: two let the next tile's MMAs run under this tile's epilogue; with one,
+    // the epilogue reads the whole accumulator into registers first and releases it at once
+    static constexpr int ACC_BUFS = ACC_BUFS_;
+    static_assert(ACC_BUFS == 1 || ACC_BUFS == 2, "accumulator buffers");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && BN_CTA % 8 == 0, "BLOCK_N");
 
     // One K step = one 128-byte swizzle row per operand row: 64 bf16, 128 E4M3, 256 E2M1.
@@ -90,9 +106,9 @@ struct GemmCfg {
     static constexpr int SFB_CHUNK = SCALED ? SFB_ATOMS * UT_WORDS * 512 : 0;
     static constexpr int SF_STAGE_BYTES = SFA_CHUNK + SFB_CHUNK;
 
-    // Tensor memory: two fp32 accumulators of BN columns, then rotating scale slots.
+    // Tensor memory: ACC_BUFS fp32 accumulators of BN columns, then rotating scale slots.
     static constexpr int TMEM_COLS = 512;
-    static constexpr int ACC_COLS = 2 * BN;
+    static constexpr int ACC_COLS = ACC_BUFS * BN;
     static constexpr int SFA_COLS = UT_WORDS * 4;
     static constexpr int SFB_COLS = UT_WORDS * SFB_ATOMS * 4;
     static constexpr int SF_SLOT_COLS = SFA_COLS + SFB_COLS;
@@ -113,6 +129,9 @@ struct GemmCfg {
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    // a K slice of a split tile is a worker's last work item, so its epilogue stages the
+    // fp32 partial sums (BM x BN) in the then idle A/B stage buffers
+    static_assert(BM * BN * 4 <= OFF_SF, "stage buffers too small for a split tile's partial sums");
 
     static constexpr int THREADS = 192;
 };
@@ -120,6 +139,22 @@ struct GemmCfg {
 struct Tile {
     int m_blk, n_blk;
 };
+
+// One work item: a tile and the K steps [kb0, kb1) it covers; `tail` >= 0 for a K slice of
+// a split tile (its index among the split tiles).
+struct Work {
+    int tile, kb0, kb1, tail, slice;
+};
+
+// Slices are cut at scale-group boundaries (`period` K steps), as evenly as the groups allow.
+__device__ __forceinline__ Work work_of(const GemmArgs& a, int w, int period) {
+    if (w < a.full_tiles) return Work{w, 0, a.num_kb, -1, 0};
+    const int u = w - a.full_tiles;
+    const int tail = u / a.splits, j = u - tail * a.splits;
+    const int groups = (a.num_kb + period - 1) / period;
+    const int g0 = j * groups / a.splits, g1 = (j + 1) * groups / a.splits;
+    return Work{a.full_tiles + tail, g0 * period, min(g1 * period, a.num_kb), tail, j};
+}
 
 __device__ __forceinline__ Tile tile_of(const GemmArgs& a, int t) {
     const int per_group = a.group_m * a.n_blocks;
@@ -183,7 +218,8 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
-                const __grid_constant__ CUtensorMap tm_d, const GemmArgs args) {
+                const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_ws,
+                const GemmArgs args) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -220,6 +256,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
         tma_prefetch_desc(&tm_d);
+        if (args.splits > 1) tma_prefetch_desc(&tm_ws);
         if constexpr (C::SCALED) {
             tma_prefetch_desc(&tm_sfa);
             tma_prefetch_desc(&tm_sfb);
@@ -247,8 +284,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int t = worker; t < args.num_tiles && ok; t += workers) {
-                const Tile tl = tile_of(args, t);
+            for (int w = worker; w < args.num_work && ok; w += workers) {
+                const Work wk = work_of(args, w, C::SF_PERIOD);
+                const Tile tl = tile_of(args, wk.tile);
                 const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
                 const int n0 = tl.n_blk * C::BN;
                 const int nb0 = n0 + (int)rank * C::BN_CTA;
@@ -260,7 +298,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         g = 0;
                     }
                 }
-                for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+                for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!bounded_wait(&empty[s], ph ^ 1u, args, abort_flag)) {
@@ -315,9 +353,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, lt = 0, git = 0;
             bool ok = true;
-            for (int t = worker; t < args.num_tiles && ok; t += workers, ++lt) {
-                const uint32_t buf = lt & 1u;
-                const uint32_t aph = (lt >> 1) & 1u;
+            for (int w = worker; w < args.num_work && ok; w += workers, ++lt) {
+                const Work wk = work_of(args, w, C::SF_PERIOD);
+                const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
+                const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
                 if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
                     ok = false;
                     break;
@@ -325,7 +364,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * C::BN;
                 uint32_t slot = 0;
-                for (int kb = 0; kb < args.num_kb; ++kb, ++it) {
+                for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!bounded_wait(&full[s], ph, args, abort_flag)) {
@@ -371,7 +410,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         // 32 bytes of K per MMA: 16 bf16, 32 E4M3, 64 E2M1
                         const uint64_t ad = adesc + (uint64_t)(2 * i);
                         const uint64_t bd = bdesc + (uint64_t)(2 * i);
-                        const uint32_t acc = (kb > 0 || i > 0) ? 1u : 0u;
+                        const uint32_t acc = (kb > wk.kb0 || i > 0) ? 1u : 0u;
                         if constexpr (C::kind == Kind::BF16) {
                             const uint32_t id = idesc_bf16(C::TILE_M, C::BN);
                             if constexpr (C::PAIR)
@@ -421,12 +460,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t quarter = warp % 4;  // TMEM lanes this warp may read
         uint8_t* epi = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BLOCK;
         uint32_t lt = 0, nblk = 0;
-        for (int t = worker; t < args.num_tiles; t += workers, ++lt) {
-            const Tile tl = tile_of(args, t);
+        for (int w = worker; w < args.num_work; w += workers, ++lt) {
+            const Work wk = work_of(args, w, C::SF_PERIOD);
+            const Tile tl = tile_of(args, wk.tile);
             const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
             const int n0 = tl.n_blk * C::BN;
-            const uint32_t buf = lt & 1u;
-            const uint32_t aph = (lt >> 1) & 1u;
+            const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
+            const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
             if (!warp_wait(&tmem_full[buf], aph, args, abort_flag)) break;
             tc_fence_after();
             const int row = m0 + (int)(quarter * 32 + lane);
@@ -440,37 +480,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
             }
             const uint32_t taddr = tmem_base + ((quarter * 32) << 16) + buf * C::BN;
-#pragma unroll 1
-            for (int c = 0; c < C::BN / 32; ++c, ++nblk) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, r);
-                tmem_ld_wait();
-                if (c == C::BN / 32 - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (leader)
-                            mbar_arrive(&tmem_empty[buf]);
-                        else
-                            mbar_arrive_remote(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
-                    }
+            const auto release = [&] {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(&tmem_empty[buf]);
+                    else
+                        mbar_arrive_remote(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
                 }
+            };
+            const auto pack = [&](uint32_t lo, uint32_t hi) -> uint32_t {
+                __nv_bfloat162 v = __float22bfloat162_rn(make_float2(__uint_as_float(lo), __uint_as_float(hi)));
+                return zero_row ? 0u : *reinterpret_cast<uint32_t*>(&v);
+            };
+            // one 32 x 32 block (16 packed bf16 pairs per lane) through the swizzled staging
+            // buffer to D
+            const auto store_block = [&](int c, const uint32_t* w16) {
                 // the store issued from this buffer two blocks ago has finished reading it
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
                 uint8_t* blk = epi + (nblk & 1u) * C::EPI_BLOCK;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {  // 16-byte chunk q of this row (8 columns)
-                    uint32_t w[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        __nv_bfloat162 v = __float22bfloat162_rn(make_float2(__uint_as_float(r[8 * q + 2 * h]),
-                                                                             __uint_as_float(r[8 * q + 2 * h + 1])));
-                        w[h] = zero_row ? 0u : *reinterpret_cast<uint32_t*>(&v);
-                    }
                     // 64-byte swizzle: chunk q of row l sits at chunk q ^ ((l >> 1) & 3)
                     const uint32_t pos = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
-                    *reinterpret_cast<uint4*>(blk + pos) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(blk + pos) =
+                        make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -478,6 +514,133 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     tma_store_2d(&tm_d, blk, n0 + c * 32, m0 + (int)quarter * 32);
                     bulk_commit_group();
                 }
+                ++nblk;
+            };
+            if (wk.tail >= 0) {
+                // K slice of a split tile (this worker's last work item: no copy or MMA touches
+                // the stage buffers any more).  Each warp lays its 32 rows of fp32 partial sums
+                // out in the stage buffers as 32 x 32 blocks (128-byte swizzle) and stores them
+                // with TMA in the slice's workspace slot.
+                const int64_t slot_stride = (int64_t)C::TILE_M * C::BN;
+                const int slot_row = (wk.tail * args.splits + wk.slice) * C::TILE_M + (int)rank * C::BM + (int)quarter * 32;
+                uint8_t* stage = smem + C::OFF_A + (warp - 2) * (32 * C::BN * 4);
+#pragma unroll 1
+                for (int c = 0; c < C::BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
+                    if (c == C::BN / 32 - 1) release();
+                    uint8_t* blk = stage + c * 4096;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {  // 16-byte chunk v of this row sits at chunk v ^ (row % 8)
+                        const uint32_t pos = lane * 128 + ((v ^ (lane & 7)) << 4);
+                        *reinterpret_cast<uint4*>(blk + pos) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    for (int c = 0; c < C::BN / 32; ++c) tma_store_2d(&tm_ws, stage + c * 4096, c * 32, slot_row);
+                    bulk_commit_group();
+                    bulk_wait_group_all();  // complete in memory, not only read
+                    fence_proxy_async_global();
+                }
+                // publish this slice, then wait (bounded) until every slice of these rows has
+                bool ok = true;
+                if (lane == 0) {
+                    __threadfence();
+                    int* cnt = args.tail_count + (wk.tail * C::CTAS + (int)rank) * 4 + (int)quarter;
+                    atomicAdd(cnt, 1);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (*reinterpret_cast<volatile int*>(cnt) < args.splits) {
+                        if (*abort_flag) {
+                            ok = false;
+                            break;
+                        }
+                        if (globaltimer_ns() - t0 > args.timeout_ns) {
+                            latch_status(args.status, kStatusTimeout);
+                            *abort_flag = 1;
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    __threadfence();
+                }
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+                // this slice's share of the 32 rows: sum the slots in order, round, store.  The
+                // (row, slot) pairs are walked four at a time with all their loads in flight.
+                const int S = args.splits;
+                const int r0 = wk.slice * 32 / S, r1 = (wk.slice + 1) * 32 / S;
+                const int col = (int)lane * 8;  // 8 columns per lane
+                const int n = n0 + col;
+                const bool col_ok = col < C::BN && n < args.N;
+                const float* base = args.ws + (int64_t)wk.tail * S * slot_stride +
+                                    (int64_t)((int)rank * C::BM + (int)quarter * 32) * C::BN + col;
+                const int pairs = (r1 - r0) * S;
+                float v[8];
+                for (int b = 0; b < pairs; b += 4) {
+                    float4 x[8];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int pi = b + u, i = r0 + pi / S, j = pi % S;
+                        if (pi < pairs && col_ok && m0 + (int)quarter * 32 + i < args.M) {
+                            const float4* p4 = reinterpret_cast<const float4*>(base + j * slot_stride + (int64_t)i * C::BN);
+                            x[2 * u] = __ldcg(p4);
+                            x[2 * u + 1] = __ldcg(p4 + 1);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int pi = b + u, i = r0 + pi / S, j = pi % S;
+                        const int row = m0 + (int)quarter * 32 + i;
+                        if (pi >= pairs || !col_ok || row >= args.M) continue;
+                        if (j == 0) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+                        }
+                        v[0] += x[2 * u].x, v[1] += x[2 * u].y, v[2] += x[2 * u].z, v[3] += x[2 * u].w;
+                        v[4] += x[2 * u + 1].x, v[5] += x[2 * u + 1].y, v[6] += x[2 * u + 1].z, v[7] += x[2 * u + 1].w;
+                        if (j != S - 1) continue;
+                        __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
+                        if (n + 8 <= args.N) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(v[2 * e], v[2 * e + 1]));
+                                o[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+                        } else {
+                            for (int e = 0; e < 8 && n + e < args.N; ++e) dst[e] = __float2bfloat16_rn(v[e]);
+                        }
+                    }
+                }
+            } else if constexpr (C::ACC_BUFS == 2) {
+#pragma unroll 1
+                for (int c = 0; c < C::BN / 32; ++c) {
+                    uint32_t r[32], w[16];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
+                    if (c == C::BN / 32 - 1) release();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) w[h] = pack(r[2 * h], r[2 * h + 1]);
+                    store_block(c, w);
+                }
+            } else {
+                // drain the whole accumulator row into registers (bf16 pairs), free it, then store
+                uint32_t w[C::BN / 2];
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) w[16 * c + h] = pack(r[2 * h], r[2 * h + 1]);
+                }
+                release();
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c) store_block(c, w + 16 * c);
             }
         }
         if (lane == 0) bulk_wait_group_all();

@@ -16,11 +16,13 @@ int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* 
 // Bytes of scratch the FP8 GEMM lays its scale chunks out in, for this problem.
 int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n);
 
-// FP8 block-scaled GEMM on packed SF words, same rules as gemm_fp8_nt; faults latch `status`;
-// the scale chunks go to `scale_scratch` (gemm_fp8_scale_scratch_bytes bytes, 256-aligned).
+// FP8 block-scaled GEMM on packed SF words, same rules as gemm_fp8_nt; faults latch `status`.
+// `scratch` (256-aligned, `scratch_bytes` >= gemm_fp8_scale_scratch_bytes) takes the scale
+// chunks and, when it has room, the workspace of a split last wave.
 int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const void* sfb, void* D, int M, int N,
                            int K, int64_t lda, int64_t ldb, int64_t ldd, int64_t ld_sfa, int64_t ld_sfb,
-                           int sfb_gran_n, int* status, void* scale_scratch, cudaStream_t stream);
+                           int sfb_gran_n, int* status, void* scratch, int64_t scratch_bytes,
+                           cudaStream_t stream);
 
 }  // namespace detail
 }  // namespace bsp

@@ -83,5 +83,6 @@ extern "C" int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const vo
     if (const int rc = bsp::detail::launch_sf_transform_u8(sfb_e8m0, mn_b, kb, ld_sfb_in, sfb_w, ld_b, status, st))
         return rc;
     return bsp::detail::launch_gemm_fp8_packed(A, sfa_w, B, sfb_w, D, M, N, K, lda, ldb, ldd, ld_a, ld_b,
-                                               sfb_gran_n, status, sfa_w + off_chunks, st);
+                                               sfb_gran_n, status, sfa_w + off_chunks,
+                                               (int64_t)kScratchBytes - off_chunks, st);
 }

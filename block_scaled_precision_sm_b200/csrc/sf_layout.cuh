@@ -61,18 +61,22 @@ __device__ __forceinline__ void sf_layout_word(const uint16_t* __restrict__ in, 
     }
 }
 
-// Both operands' chunks in one launch: words [0, total_a) of A, then those of B.
+// Both operands' chunks in one launch: words [0, total_a) of A, then those of B, then
+// `zero_vecs` 16-byte zeros at `zero` (the GEMM's split-tail counters and workspace).
 __global__ void __launch_bounds__(256) sf_tmem_layout_kernel(const uint16_t* __restrict__ in_a, SfLayout pa,
                                                              uint32_t* __restrict__ out_a,
                                                              const uint16_t* __restrict__ in_b, SfLayout pb,
-                                                             uint32_t* __restrict__ out_b) {
-    const int64_t na = sf_layout_words(pa), total = na + sf_layout_words(pb);
+                                                             uint32_t* __restrict__ out_b, uint4* __restrict__ zero,
+                                                             int64_t zero_vecs) {
+    const int64_t na = sf_layout_words(pa), nab = na + sf_layout_words(pb), total = nab + zero_vecs;
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         if (idx < na)
             sf_layout_word(in_a, pa, out_a, idx);
-        else
+        else if (idx < nab)
             sf_layout_word(in_b, pb, out_b, idx - na);
+        else
+            zero[idx - nab] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 

@@ -180,6 +180,21 @@ const char* bsp_status_string(int status);
 uint64_t bsp_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * bsp_gemm_plan — how a GEMM of this kind and shape would be launched on the current
+ * device, without launching it.  kind: 0 BF16, 1 FP8 (gemm_fp8_nt), 2 FP4, 3 M-grouped FP8
+ * (M = M_total).  Writes six int32 to `plan` (caller-owned host memory):
+ *   plan[0] rows per tile (128 single CTA, 256 CTA pair)   plan[1] columns per tile
+ *   plan[2] K slices per split tile (1: no split)          plan[3] split tiles
+ *   plan[4] work items (whole tiles + slices)              plan[5] persistent workers launched
+ * The tiles left after the last full wave of workers are cut along K into slices at
+ * scale-group boundaries when that shortens the last wave (at least two slices of eight or
+ * more K steps); their fp32 partial sums meet in a workspace and are added in slice order
+ * before the bf16 rounding, so results do not change from run to run.
+ * Returns BSP_ERR_ARG for a bad kind, sizes <= 0 or a NULL plan; needs an sm_100 device.
+ */
+int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan);
+
+/*
  * bsp_kernel_launches — number of kernels this library has launched in this process
  * (all devices, all calls).  For the bench's launch count.
  */

@@ -79,6 +79,16 @@ def test_rejects_bad_arguments_without_gpu(lib):
     assert lib.transform_sf_ue8m0(good, 1, 64, 8, 8, vp(0x10010), 64, None) == -1
 
 
+def test_plan_rejects_bad_arguments_without_gpu(lib):
+    plan = (ctypes.c_int32 * 6)()
+    ptr = ctypes.cast(plan, ctypes.c_void_p)
+    assert lib.bsp_gemm_plan(4, 256, 256, 256, ptr) == -1  # no such kind
+    assert lib.bsp_gemm_plan(-1, 256, 256, 256, ptr) == -1
+    assert lib.bsp_gemm_plan(1, 0, 256, 256, ptr) == -1
+    assert lib.bsp_gemm_plan(1, 256, 256, -128, ptr) == -1
+    assert lib.bsp_gemm_plan(1, 256, 256, 256, None) == -1
+
+
 def test_product_path_fails_loudly_without_library(tmp_path, monkeypatch):
     from block_scaled_precision_sm_b200 import _lib
 

@@ -188,6 +188,70 @@ def test_fp4(ops, orc, m, n, k):
     check_gemm(bf16_to_f64(D), orc.gemm_fp4(p["A"], p["sfa"], p["B"], p["sfb"]), f"fp4 {m}x{n}x{k}")
 
 
+# ------------------------------------------------------------------ split last wave
+
+def _run_kind(ops, kind, m, n, k, seed, gran=128, rows=None, cols=None):
+    """Run one GEMM on the GPU and return (D as f64, oracle value on rows x cols)."""
+    ldd = (n + 7) // 8 * 8
+    D = torch.empty((m, ldd), dtype=torch.bfloat16, device="cuda")[:, :n]
+    orc_args = dict(rows=rows, cols=cols) if rows is not None else {}
+    if kind == "fp8":
+        p = inputs.dense_fp8_problem(m, n, k, seed=seed, b_block_rows=gran)
+        ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]), D, sfb_gran_n=gran)
+        ref = lambda orc: orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"], gran_n=gran, **orc_args)
+    elif kind == "fp4":
+        p = inputs.dense_fp4_problem(m, n, k, seed=seed)
+        ops.gemm_fp4_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]), D)
+        ref = lambda orc: orc.gemm_fp4(p["A"], p["sfa"], p["B"], p["sfb"], **orc_args)
+    else:
+        p = inputs.dense_bf16_problem(m, n, k, seed=seed)
+        ops.gemm_bf16_nt(to_dev(p["A"], torch.bfloat16), to_dev(p["B"], torch.bfloat16), D)
+        ref = lambda orc: orc.gemm_bf16(p["A"], p["B"], **orc_args)
+    _status_ok(ops)
+    got = bf16_to_f64(D)
+    if rows is not None:
+        got = got[np.ix_(rows, cols)]
+    return got, ref
+
+
+# Shapes whose tiles are fewer than the workers: every tile is cut along K into slices whose
+# fp32 partial sums are added in a workspace; ragged M / N, uneven slices (K = 2560: five
+# scale groups in two slices) and a partial last scale group (K = 2688) included.
+@pytest.mark.parametrize("kind,m,n,k,gran", [("fp8", 256, 1024, 4096, 128), ("fp8", 300, 1000, 2560, 128),
+                                             ("fp8", 300, 1000, 2688, 1), ("bf16", 256, 512, 4096, 1),
+                                             ("bf16", 130, 1000, 4096, 1), ("fp4", 256, 512, 8192, 1)])
+def test_split_tiles_every_output(ops, orc, kind, m, n, k, gran):
+    plan = ops.gemm_plan(kind, m, n, k)
+    assert plan["splits"] > 1 and plan["split_tiles"] * plan["splits"] == plan["work_items"], plan
+    got, ref = _run_kind(ops, kind, m, n, k, seed=m + k, gran=gran)
+    check_gemm(got, ref(orc), f"{kind} split {m}x{n}x{k} {plan}")
+
+
+# More tiles than workers: whole tiles in full waves, the remainder split; the oracle checks a
+# sample of rows and columns that meets every tile.
+@pytest.mark.parametrize("kind,m,n,k", [("fp8", 2560, 2048, 2048), ("bf16", 2560, 2048, 1024),
+                                        ("fp4", 2560, 2048, 4096)])
+def test_split_last_wave_sampled(ops, orc, kind, m, n, k):
+    plan = ops.gemm_plan(kind, m, n, k)
+    assert plan["splits"] > 1 and plan["work_items"] > plan["split_tiles"] * plan["splits"], plan
+    rng = np.random.default_rng(k)
+    tm, tn = plan["tile_m"], plan["tile_n"]
+    rows = np.unique(np.concatenate([rng.integers(r, min(r + tm, m), 6) for r in range(0, m, tm)])).astype(np.int32)
+    cols = np.unique(np.concatenate([rng.integers(c, min(c + tn, n), 6) for c in range(0, n, tn)])).astype(np.int32)
+    got, ref = _run_kind(ops, kind, m, n, k, seed=7, rows=rows, cols=cols)
+    check_gemm(got, ref(orc), f"{kind} last wave {m}x{n}x{k} {plan}")
+
+
+def test_split_is_deterministic(ops):
+    # slices are added in a fixed order, so repeated runs give identical bytes
+    p = inputs.dense_fp8_problem(256, 1024, 4096, seed=5)
+    args = [to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")]
+    d1 = ops.gemm_fp8_nt(*args)
+    d2 = ops.gemm_fp8_nt(*args)
+    _status_ok(ops)
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
 # ------------------------------------------------------------------ grouped
 
 def _grouped(ops, p):
@@ -235,16 +299,21 @@ def test_grouped_bad_index_is_flagged(ops):
 # ------------------------------------------------------------------ failure detection
 
 def test_wait_timeout_is_reported_and_context_survives(ops, orc):
-    # a 2 us wait limit cannot hold a K=8192 tile: a wait runs out, the kernel winds down
-    p = inputs.dense_fp8_problem(512, 448, 8192, seed=4)
-    args = [to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")]
+    # a 2 us wait limit cannot hold whole 256 x 256 x 8192 tiles (40 tiles: too many to split
+    # along K): the epilogue's wait for the accumulator runs out and the kernel winds down
+    m, n, k = 1280, 2048, 8192
+    assert ops.gemm_plan("fp8", m, n, k)["splits"] == 1
+    big = inputs.dense_fp8_problem(m, n, k, seed=4)
+    args = [to_dev(big[x]) for x in ("A", "sfa", "B", "sfb")]
     old = ops.set_wait_timeout_ns(2000)
     try:
         ops.gemm_fp8_nt(*args)
         assert ops.device_status() == -6
     finally:
         ops.set_wait_timeout_ns(old)
-    D = ops.gemm_fp8_nt(*args)
+    # the context is still usable
+    p = inputs.dense_fp8_problem(256, 448, 1024, seed=5)
+    D = ops.gemm_fp8_nt(*[to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")])
     _status_ok(ops)
     check_gemm(bf16_to_f64(D), orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"]), "after timeout")
 
