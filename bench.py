@@ -260,6 +260,7 @@ def run_ours(args):
     fp8_peak = peaks["bf16_tflops"] * NOMINAL_RATIO["fp8"]
     achieved = flops / (gemm_ms * 1e-3) / 1e12
     traffic = profiled_traffic("gemm_fp8_4096x7168x16384.md")
+    plan = ops.gemm_plan("fp8", M, N, K)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -276,7 +277,8 @@ def run_ours(args):
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
                      "frac_of_sustained": round(achieved / (peaks.get("bf16_tflops_sustained", 1400.0) * 2), 4),
-                     "kernel": "gemm_kernel<FP8,224>", "kernel_ms": round(gemm_ms, 5)},
+                     "kernel": "gemm_kernel<FP8, {tile_m}x{tile_n} pair tiles>".format(**plan),
+                     "plan": plan, "kernel_ms": round(gemm_ms, 5)},
         "gpu_launches": int(launches),
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 3),

@@ -204,16 +204,20 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     a.timeout_ns = g_timeout_ns.load();
     const int workers = a.num_work < max_workers ? a.num_work : max_workers;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C::CTAS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Scaled kinds follow their own scale layout pass on the stream: the GEMM may launch while
+    // that pass runs (set-up, operand loads) and waits for it only before reading its output.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = C::SCALED ? 2 : 1;
     cfg.gridDim = dim3(C::CTAS * workers);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, td, tw, a);
     g_launches.fetch_add(1);
@@ -310,6 +314,11 @@ int launch_sf_layout(const void* in_a, const SfLayout& pa, void* out_a, const vo
 // mapped between calls (the default pool would hand it back to the driver at every
 // synchronisation and map it again on the next call).
 int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+    // under stream capture the allocation becomes a graph memory node (graph-owned pool)
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return BSP_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusActive)
+        return cudaMallocAsync(p, bytes, stream) == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
     static std::mutex mu;
     static cudaMemPool_t pools[kMaxDevices] = {};
     int dev = 0;

@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
+            bool prior_done = false;  // the scale chunks come from the kernel launched before
             for (int w = worker; w < args.num_work && ok; w += workers) {
                 const Work wk = work_of(args, w, C::SF_PERIOD);
                 const Tile tl = tile_of(args, wk.tile);
@@ -315,6 +316,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
                     const int q = kb / C::SF_PERIOD;
+                    if (sf_here && !prior_done) {
+                        griddep_wait();
+                        prior_done = true;
+                    }
                     if constexpr (C::PAIR) {
                         const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), 0);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
@@ -549,6 +554,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 bool ok = true;
                 if (lane == 0) {
                     __threadfence();
+                    griddep_wait();  // the counters were zeroed by the kernel launched before
                     int* cnt = args.tail_count + (wk.tail * C::CTAS + (int)rank) * 4 + (int)quarter;
                     atomicAdd(cnt, 1);
                     const uint64_t t0 = globaltimer_ns();

@@ -102,6 +102,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
+// start while the kernel before it still runs; griddep_wait blocks the calling thread until
+// that kernel has completed and its writes are visible (it returns at once otherwise), and
+// griddep_launch_dependents lets the next kernel start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Orders this thread's async-proxy global accesses (completed bulk copies) with its later
 // generic-proxy ones.
 __device__ __forceinline__ void fence_proxy_async_global() {

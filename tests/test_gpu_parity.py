@@ -252,6 +252,31 @@ def test_split_is_deterministic(ops):
     assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
 
 
+def test_cuda_graph_capture_replays_the_same_bytes(ops):
+    # the calls are capturable: scratch becomes a graph memory node, launches become kernel
+    # nodes; a replay on new inputs (copied into the captured buffers) matches an eager call
+    p = inputs.dense_fp8_problem(512, 1024, 4096, seed=21)
+    q = inputs.dense_fp8_problem(512, 1024, 4096, seed=22)
+    dv = {x: to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")}
+    sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
+    D = torch.empty((512, 1024), dtype=torch.bfloat16, device="cuda")
+    ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # first call outside capture sets the kernels up
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.transform_sf_ue8m0(dv["sfa"], out=sa)
+        ops.transform_sf_ue8m0(dv["sfb"], out=sb)
+        ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)
+    for x in ("A", "sfa", "B", "sfb"):
+        dv[x].copy_(to_dev(q[x]))
+    g.replay()
+    torch.cuda.synchronize()
+    _status_ok(ops)
+    eager = ops.gemm_fp8_nt(*[to_dev(q[x]) for x in ("A", "sfa", "B", "sfb")])
+    _status_ok(ops)
+    assert torch.equal(D.view(torch.int16), eager.view(torch.int16))
+
+
 # ------------------------------------------------------------------ grouped
 
 def _grouped(ops, p):
