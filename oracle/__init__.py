@@ -166,3 +166,18 @@ def gemm_grouped_fp8(A, sfa, B, sfb, m_indices, gran_n=128, rows=None, cols=None
                                        _p(r), nr, _p(c), nc, _p(out)):
         raise ValueError("gemm_grouped_fp8: bad arguments (expert index out of range?)")
     return out
+
+
+def quantize_fp8(x, block_rows: int = 1):
+    """fp32 (or bf16 bit patterns, uint16) [R, K] -> (E4M3 codes uint8 [R, K],
+    biased UE8M0 bytes uint8 [ceil(R/block_rows), K/128]); blocks of block_rows x 128."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        x = (x.astype(np.uint32) << 16).view(np.float32)
+    x = _c(x, np.float32)
+    r, k = x.shape
+    q = np.empty((r, k), np.uint8)
+    e = np.empty((-(-r // block_rows), k // 128), np.uint8)
+    if _load().oracle_quantize_fp8(_p(x), r, k, ctypes.c_int64(k), block_rows, _p(q), _p(e)):
+        raise ValueError("quantize_fp8: bad sizes or a non-finite value")
+    return q, e

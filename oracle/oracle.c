@@ -23,6 +23,13 @@
  *        16-bit word, stored MN-major: out[j*ld + mn] = e[mn][2j] | e[mn][2j+1] << 8.
  *        Reading (the pages give no byte order): the lower K block sits in the
  *        low byte; mn >= MN and the missing high byte of an odd count are 0.
+ *   Quantiser ("Fatores de escala FP8 e o formato UE8M0" on the crazystack page:
+ *        one power-of-two scale per block, so that the block fits the FP8 range):
+ *        per block of block_rows x 128 values, e = the smallest integer with
+ *        448 * 2^e >= max |x| (0 for an all-zero block), clamped to [-126, 127],
+ *        stored as the UE8M0 byte e + 127; each value becomes x / 2^e rounded to
+ *        the nearest E4M3 value, ties to the even code, sign kept (also for a
+ *        zero result), magnitudes above 448 saturated.
  *
  * Decode tables are built from each format's bit fields (sign, exponent,
  * mantissa), not typed in.  For FP8 every product has at most 8 significant
@@ -258,6 +265,74 @@ int oracle_gemm_grouped_fp8(const uint8_t* A, const uint8_t* sfa, const uint8_t*
                             sbg + (int64_t)(n / gran_n) * KB, K);
             }
             out[(int64_t)i * C + j] = v;
+        }
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------------- quantiser */
+
+/* Smallest integer e with qmax * 2^e >= amax (0 for amax == 0): an exact search
+ * upward from a start at least one binade too low. */
+static int exponent_for_amax(double amax, double qmax) {
+    if (amax == 0.0) return 0;
+    int ex, eq;
+    frexp(amax, &ex); /* amax in [2^(ex-1), 2^ex) */
+    frexp(qmax, &eq); /* qmax in [2^(eq-1), 2^eq) */
+    int e = ex - eq - 1;
+    while (ldexp(qmax, e) < amax) ++e;
+    return e;
+}
+
+/* Finite v -> E4M3 (FN) code, round to nearest with ties to the even code.  The value
+ * grid of a binade [2^E, 2^(E+1)) has spacing 2^(E-3) for E >= -6 and 2^-9 below
+ * (subnormals), so rint(|v| / spacing) picks the nearest grid point and rint's ties go
+ * to the even integer, which is the even mantissa. */
+static uint8_t encode_e4m3_rne(double v) {
+    unsigned s = signbit(v) ? 0x80u : 0u;
+    double a = fabs(v);
+    int ex;
+    frexp(a, &ex);
+    int E = ex - 1;
+    double step = (a == 0.0 || E < -6) ? ldexp(1.0, -9) : ldexp(1.0, E - 3);
+    double r = rint(a / step) * step;
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return (uint8_t)s;
+    frexp(r, &ex);
+    E = ex - 1;
+    unsigned code;
+    if (E < -6)
+        code = (unsigned)(r / ldexp(1.0, -9)); /* exponent field 0, mantissa 1..7 */
+    else
+        code = ((unsigned)(E + 7) << 3) | (unsigned)((r / ldexp(1.0, E) - 1.0) * 8.0);
+    return (uint8_t)(s | code);
+}
+
+/* x [rows][ld_x] fp32 -> q [rows][cols] E4M3 codes and e [ceil(rows/block_rows)][cols/128]
+ * biased UE8M0 bytes.  Returns -1 for bad sizes or a non-finite input. */
+int oracle_quantize_fp8(const float* x, int rows, int cols, int64_t ld_x, int block_rows, uint8_t* q,
+                        uint8_t* e) {
+    if (rows < 0 || cols < 0 || cols % 128 || block_rows < 1 || ld_x < cols) return -1;
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < cols; ++c)
+            if (!isfinite(x[(int64_t)r * ld_x + c])) return -1;
+    int KB = cols / 128, RB = (rows + block_rows - 1) / block_rows;
+    for (int rb = 0; rb < RB; ++rb) {
+        int r0 = rb * block_rows, r1 = r0 + block_rows < rows ? r0 + block_rows : rows;
+        for (int kb = 0; kb < KB; ++kb) {
+            double amax = 0.0;
+            for (int r = r0; r < r1; ++r)
+                for (int c = kb * 128; c < kb * 128 + 128; ++c) {
+                    double a = fabs((double)x[(int64_t)r * ld_x + c]);
+                    if (a > amax) amax = a;
+                }
+            int ex = exponent_for_amax(amax, 448.0);
+            if (ex < -126) ex = -126;
+            if (ex > 127) ex = 127;
+            e[(int64_t)rb * KB + kb] = (uint8_t)(ex + 127);
+            for (int r = r0; r < r1; ++r)
+                for (int c = kb * 128; c < kb * 128 + 128; ++c)
+                    q[(int64_t)r * cols + c] = encode_e4m3_rne(ldexp((double)x[(int64_t)r * ld_x + c], -ex));
         }
     }
     return 0;

@@ -27,6 +27,14 @@ MUTANTS = {
     "sf_pack_byte_order": ("v = (uint16_t)(lo | (hi << 8));", "v = (uint16_t)(hi | (lo << 8));"),
     "bf16_truncates": ("q = ldexp(rint(ldexp(x, -lsb)), lsb);", "q = ldexp(trunc(ldexp(x, -lsb)), lsb);"),
     "padding_rows_use_expert0": ("int g = m_indices[m];", "int g = m_indices[m] < 0 ? 0 : m_indices[m];"),
+    "quant_exponent_one_low": ("while (ldexp(qmax, e) < amax) ++e;", "while (ldexp(qmax, e + 1) < amax) ++e;"),
+    "quant_truncates": ("double r = rint(a / step) * step;", "double r = trunc(a / step) * step;"),
+    "quant_ties_away": ("double r = rint(a / step) * step;", "double r = round(a / step) * step;"),
+    "quant_drops_sign": ("unsigned s = signbit(v) ? 0x80u : 0u;", "unsigned s = v < 0.0 ? 0x80u : 0u;"),
+    "quant_block_first_row_only": ("for (int r = r0; r < r1; ++r)\n                for (int c = kb * 128; c < kb * 128 + 128; ++c) {\n                    double a",
+                                   "for (int r = r0; r < r0 + 1; ++r)\n                for (int c = kb * 128; c < kb * 128 + 128; ++c) {\n                    double a"),
+    "quant_no_clamp": ("if (ex < -126) ex = -126;", "if (ex < -127) ex = -127;"),
+    "quant_subnormal_step": ("ldexp(1.0, -9) : ldexp(1.0, E - 3);", "ldexp(1.0, -10) : ldexp(1.0, E - 3);"),
     "bf16_sign": ("acc += decode_bf16(A[(int64_t)m * K + k]) * decode_bf16(B[(int64_t)n * K + k]);",
                   "acc -= decode_bf16(A[(int64_t)m * K + k]) * decode_bf16(B[(int64_t)n * K + k]);"),
 }

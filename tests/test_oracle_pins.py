@@ -7,7 +7,10 @@
   ml_dtypes) on tiny shapes, and against closed forms (identity, all-ones,
   single non-unit scale);
 * the SF packing against a hand-worked example and the pack/unpack round trip;
-* the bf16 rounding against brute-force nearest-even over all bf16 values.
+* the bf16 rounding against brute-force nearest-even over all bf16 values;
+* the quantiser against ml_dtypes' E4M3 rounding, the defining inequality of the
+  block exponent, hand-worked blocks (ties, subnormals, signed zeros, the clamp)
+  and the input generator's independent numpy quantiser.
 """
 
 from fractions import Fraction
@@ -316,3 +319,95 @@ def test_sampled_equals_full(orc):
     rows, cols = np.array([0, 63, 17]), np.array([95, 0, 40, 41])
     assert np.array_equal(orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"], rows=rows, cols=cols),
                           full[np.ix_(rows, cols)])
+
+
+# ---------------------------------------------------------------- quantiser
+
+def _quant_data(rows, cols, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    # spread the block magnitudes over many binades, including tiny and huge ones
+    rs = np.ldexp(np.float32(1.0), rng.integers(-60, 60, size=(rows, 1))).astype(np.float32)
+    x = (x * rs).astype(np.float32)
+    x[0, :128] = 0.0                      # an all-zero block
+    x[1 % rows, 5] = -0.0
+    x[-1, -128:] *= np.float32(2.0 ** -100)  # a block below the clamp (e < -126)
+    return x
+
+
+@pytest.mark.parametrize("block_rows,rows", [(1, 37), (128, 300), (128, 128)])
+def test_quantize_matches_ml_dtypes_rounding(orc, block_rows, rows):
+    x = _quant_data(rows, 384, seed=rows)
+    q, e = orc.quantize_fp8(x, block_rows)
+    exp = e.astype(np.int32) - 127
+    scale = np.repeat(np.repeat(np.ldexp(1.0, -exp), block_rows, axis=0)[:rows], 128, axis=1)
+    scaled = (x.astype(np.float64) * scale).astype(np.float32)  # exact: powers of two, no underflow here
+    ref = scaled.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(q, ref)
+
+
+@pytest.mark.parametrize("block_rows", [1, 128])
+def test_quantize_exponent_is_the_smallest_that_fits(orc, block_rows):
+    x = _quant_data(260, 256, seed=block_rows)
+    _, e = orc.quantize_fp8(x, block_rows)
+    rb = -(-260 // block_rows)
+    pad = np.zeros((rb * block_rows - 260, 256), np.float32)
+    amax = np.abs(np.concatenate([x, pad])).astype(np.float64).reshape(rb, block_rows, 2, 128).max(axis=(1, 3))
+    ex = e.astype(np.int64) - 127
+    free = (amax > 0) & (ex > -126)          # not zero, not clamped
+    assert np.all(448.0 * np.ldexp(1.0, ex) >= amax)
+    assert np.all(448.0 * np.ldexp(1.0, ex[free] - 1) < amax[free])
+    assert np.all(e[amax == 0] == 127)
+    assert np.all(e[(amax > 0) & (amax < 448.0 * 2.0 ** -127)] == 1)  # clamped at the UE8M0 floor
+
+
+def test_quantize_hand_blocks(orc):
+    x = np.zeros((4, 128), np.float32)
+    # row 0: amax exactly 448 * 2^3 -> e = 3, 448 * 2^3 -> 448 (0x7E); ties in units of 2^3
+    x[0, 0] = 448.0 * 8
+    x[0, 1] = (1.0 + 1.0 / 16) * 8   # halfway 1 .. 1.125 -> even mantissa 0: 1.0 = 0x38
+    x[0, 2] = (1.0 + 3.0 / 16) * 8   # halfway 1.125 .. 1.25 -> even mantissa 2: 1.25 = 0x3A
+    x[0, 3] = -(2.0 ** -10) * 8      # halfway 0 .. 2^-9 -> 0, sign kept: 0x80
+    x[0, 4] = (3.0 * 2.0 ** -10) * 8  # halfway 2^-9 .. 2^-8 -> even: 2^-8 = 0x02
+    x[0, 5] = (15.5 / 8) * 8 * 2.0 ** 7  # 1.9375 * 2^7 * 2^3: halfway 1.875..2 (binade 7) -> 2^8 = 0x78
+    # row 1: amax just above 448 -> e = 1, and 448.0 * (1 + 2^-20) / 2 -> 224 (0x76)
+    x[1, 0] = 448.0 * (1 + 2.0 ** -20)
+    # row 2: all zero, one negative zero -> byte 127, codes 0x00 / 0x80
+    x[2, 7] = -0.0
+    # row 3: amax 1.0 -> smallest e with 448 * 2^e >= 1 is -8 (448/256 = 1.75)
+    x[3, 0] = 1.0
+    x[3, 1] = -0.5
+    q, e = orc.quantize_fp8(x, 1)
+    assert list(e[:, 0]) == [130, 128, 127, 119]
+    assert list(q[0, :6]) == [0x7E, 0x38, 0x3A, 0x80, 0x02, 0x78]
+    assert q[1, 0] == 0x76
+    assert q[2, 7] == 0x80 and not q[2, :7].any() and not q[2, 8:].any()
+    # row 3: 1.0 * 2^8 = 256 = 1.0 * 2^8 -> exponent field 15, mantissa 0 = 0x78; -0.5 * 2^8 = -128 -> 0xF0
+    assert q[3, 0] == 0x78 and q[3, 1] == 0xF0
+
+
+def test_quantize_bf16_input_is_its_exact_fp32_value(orc):
+    rng = np.random.default_rng(3)
+    bits = rng.standard_normal((8, 256)).astype(np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
+    f32 = (bits.astype(np.uint32) << 16).view(np.float32)
+    for br in (1, 128):
+        qa, ea = orc.quantize_fp8(bits, br)
+        qb, eb = orc.quantize_fp8(f32, br)
+        assert np.array_equal(qa, qb) and np.array_equal(ea, eb)
+
+
+def test_quantize_rejects_non_finite(orc):
+    x = np.ones((2, 128), np.float32)
+    x[1, 3] = np.inf
+    with pytest.raises(ValueError):
+        orc.quantize_fp8(x, 1)
+
+
+@pytest.mark.parametrize("block_rows", [1, 128])
+def test_quantize_agrees_with_the_input_generator(orc, block_rows):
+    import inputs
+
+    x = np.random.default_rng(11).standard_normal((300, 512)).astype(np.float32)
+    q, e = orc.quantize_fp8(x, block_rows)
+    q2, e2 = inputs.quantize_e4m3_blocks(x, block_rows)
+    assert np.array_equal(q, q2) and np.array_equal(e, e2)
