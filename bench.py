@@ -9,7 +9,9 @@ The L2 is flushed (1 GiB write) before every timed step; the flush is outside th
 The same line also reports, each measured the same way (W warm-up, flushed L2, CUDA
 events on the launching stream): BF16 dense at the same shape, FP4 E2M1 at the same
 shape, the M-grouped FP8 MoE workload (32 experts, 32768 rows, N=4096, K=7168), the FP8
-M sweep {128, 1024, 4096} at N=K=7168, and the scale transform alone (GB/s).
+M sweep {128, 1024, 4096} at N=K=7168, the scale transform alone (GB/s), and the FP8
+quantiser that produces the GEMM's operands (fp32 A in 1x128 blocks, bf16 B in 128x128
+blocks, GB/s).
 
 FLOP convention 2*M*N*K per GEMM (the pages' own timings reproduce their TFLOPS with it).
 
@@ -44,9 +46,13 @@ PAGES_FP8_TFLOPS = 861.0   # pages' FP8xFP8 figure at this shape (Ascend 950DT):
 PAGES_BF16_TFLOPS = 431.0
 NOMINAL_RATIO = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}  # dense tensor peak relative to bf16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["block_scaled_precision_sm_b200/csrc/gemm.cuh", "block_scaled_precision_sm_b200/csrc/ptx.cuh",
-                  "block_scaled_precision_sm_b200/csrc/sf_layout.cuh", "block_scaled_precision_sm_b200/csrc/sf_transform.cuh",
-                  "block_scaled_precision_sm_b200/csrc/api.cu"]
+_CSRC = "block_scaled_precision_sm_b200/csrc/"
+# the sources each profiled kernel depends on (device code and the host code that launches it)
+KERNEL_SOURCES = {
+    "gemm": [_CSRC + f for f in ("gemm.cuh", "ptx.cuh", "sf_layout.cuh", "api.cu")],
+    "sf_transform": [_CSRC + f for f in ("sf_transform.cuh", "api.cu")],
+    "quantize": [_CSRC + f for f in ("quantize.cuh", "quantize.cu")],
+}
 
 
 def gemm_flops(m: int, n: int, k: int) -> float:
@@ -60,7 +66,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only-headline", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "sf_transform"],
+    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "sf_transform", "quantize_act",
+                                          "quantize_wgt"],
                     help="launch only this kernel (warm-up + steps launches, no timing) for an ncu capture")
     return ap.parse_args()
 
@@ -99,9 +106,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def sources_digest() -> str:
+def sources_digest(kind: str = "gemm") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -115,7 +122,8 @@ def profiled_traffic(name: str):
     txt = open(p).read()
     t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     s = re.search(r"sources_digest:\s*([0-9a-f]+)", txt)
-    if not t or not s or s.group(1) != sources_digest():
+    kind = "quantize" if name.startswith("quantize") else "sf_transform" if name.startswith("sf_transform") else "gemm"
+    if not t or not s or s.group(1) != sources_digest(kind):
         return None
     return float(t.group(1))
 
@@ -436,6 +444,31 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
                                          "bytes": int(moved), "hbm_peak_gbs": peaks["hbm_gbs"],
                                          "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                          "traffic": profiled_traffic("sf_transform_fp32_36864x56.md")}
+    del s32, w
+
+    # the quantiser (the step before the GEMM): the headline's A as fp32 in 1x128 blocks and its
+    # B as bf16 in 128x128 blocks, values -> E4M3 codes + packed UE8M0 words
+    for name, rows, bf16, br in (("quantize_fp8_fp32_4096x16384_1x128", M, False, 1),
+                                 ("quantize_fp8_bf16_7168x16384_128x128", N, True, 128)):
+        xh = inputs.normal_matrix(rows, K, seed=60 + rows, bf16=bf16)
+        x = torch.from_numpy(xh).cuda()
+        x = x.view(torch.bfloat16) if bf16 else x
+        del xh
+        qx, sx = ops.quantize_fp8(x, br)
+
+        def f_q(ev, x=x, qx=qx, sx=sx, br=br):
+            if ev is not None:
+                ev[0].record()
+            ops.quantize_fp8(x, br, q=qx, sf=sx)
+            if ev is not None:
+                ev[1].record()
+
+        ms = float(timer.run(f_q, args.warmup, reps)[:, 0].mean())
+        moved = x.numel() * x.element_size() + qx.numel() + sx.numel() * 2
+        out[name] = {"gbs": round(moved / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 5), "bytes": int(moved),
+                     "hbm_peak_gbs": peaks["hbm_gbs"], "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "traffic": profiled_traffic(name + ".md")}
+        del x, qx, sx
     return out
 
 
@@ -525,6 +558,14 @@ def run_profile(args):
         sb = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(g["sfb"][e]).cuda()) for e in range(32)])
         D = torch.empty((g["M"], 4096), dtype=torch.bfloat16, device="cuda")
         fn = lambda: ops.m_grouped_gemm_fp8_nt_contiguous(dg["A"], sa, dg["B"], sb, dg["m_indices"], D)  # noqa
+    elif args.profile in ("quantize_act", "quantize_wgt"):
+        act = args.profile == "quantize_act"
+        xh = inputs.normal_matrix(M if act else N, K, seed=60 + (M if act else N), bf16=not act)
+        x = torch.from_numpy(xh).cuda()
+        x = x if act else x.view(torch.bfloat16)
+        br = 1 if act else 128
+        qx, sx = ops.quantize_fp8(x, br)
+        fn = lambda: ops.quantize_fp8(x, br, q=qx, sf=sx)  # noqa: E731
     else:
         g = inputs.grouped_fp8_problem(32, 32768, 4096, 7168, seed=8)
         s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()

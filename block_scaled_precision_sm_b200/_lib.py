@@ -23,6 +23,7 @@ SIGNATURES = {
     "bsp_set_wait_timeout_ns": (_u64, [_u64]),
     "bsp_kernel_launches": (_u64, []),
     "bsp_gemm_plan": (_i, [_i, _i, _i, _i, _vp]),
+    "quantize_fp8_ue8m0": (_i, [_vp, _i, _i, _i, _i64, _i, _vp, _i64, _vp, _i64, _vp]),
 }
 
 STATUS = {0: "BSP_OK", -1: "BSP_ERR_ARG", -2: "BSP_ERR_ALIGN", -3: "BSP_ERR_SHAPE", -4: "BSP_ERR_UNSUPPORTED",

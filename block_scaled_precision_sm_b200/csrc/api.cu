@@ -468,6 +468,15 @@ int device_facts_noalloc(int* sms) {
 
 namespace detail {
 
+int status_word(int** out) {
+    DeviceCtx* ctx;
+    BSP_TRY(ensure_ctx(&ctx));
+    *out = ctx->status;
+    return BSP_OK;
+}
+
+void note_launch() { g_launches.fetch_add(1); }
+
 int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
                            cudaStream_t stream) {
     const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));

@@ -9,6 +9,11 @@
 namespace bsp {
 namespace detail {
 
+// The current device's status word (allocated on first use) and the launch counter of
+// bsp_kernel_launches, for entry points outside api.cu.
+int status_word(int** out);
+void note_launch();
+
 // SF words from uint8 UE8M0 bytes [mn][ld_in] into int16 [ceil(kb/2)][ld_out]; faults latch `status`.
 int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
                            cudaStream_t stream);

@@ -176,6 +176,29 @@ def kernel_launches() -> int:
     return int(_lib.load().bsp_kernel_launches())
 
 
+def quantize_fp8(x: torch.Tensor, block_rows: int = 1, q: torch.Tensor | None = None,
+                 sf: torch.Tensor | None = None, stream=None):
+    """fp32 / bf16 [rows, cols] -> (E4M3 codes uint8 [rows, cols], SF words int16
+    [ceil(cols/256), ld]) with one UE8M0 scale per block_rows x 128 block (1 or 128)."""
+    if x.dtype == torch.float32:
+        kind = 0
+    elif x.dtype == torch.bfloat16:
+        kind = 1
+    else:
+        raise ValueError("x must be float32 or bfloat16")
+    ld_x = _rowmajor(x, "x")
+    rows, cols = x.shape
+    scale_rows = -(-rows // block_rows)
+    words = (cols // 128 + 1) // 2
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty((words, sf_ld(scale_rows)), dtype=torch.int16, device=x.device)
+    _lib.call("quantize_fp8_ue8m0", _ptr(x), kind, rows, cols, ld_x, block_rows, _ptr(q), _rowmajor(q, "q"),
+              _ptr(sf), _rowmajor(sf, "sf"), _stream(stream))
+    return q, sf
+
+
 _PLAN_KINDS = {"bf16": 0, "fp8": 1, "fp4": 2, "grouped_fp8": 3}
 
 

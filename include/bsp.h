@@ -130,6 +130,31 @@ int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t l
                        void* sf_out, int64_t ld_out, void* stream);
 
 /*
+ * quantize_fp8_ue8m0 — the step before the GEMM: real values to E4M3 codes with one
+ * power-of-two UE8M0 scale per block, the scales written straight into the SF-word layout
+ * ("DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Fatores de escala FP8
+ * e o formato UE8M0 no Ascend": a power-of-two scale per block so that the block fits the
+ * FP8 range, stored as UE8M0 and packed in pairs along K, MN-major).
+ *   x [rows][ld_x]: in_kind 0 fp32, 1 bf16; all values finite (a non-finite value latches
+ *     BSP_ERR_DEVICE_CHECK; its block's codes are then unspecified).
+ *   block_rows 1: a block is 1 x 128 (activations; scale rows = rows);
+ *   block_rows 128: a block is 128 x 128 (weights; scale rows = ceil(rows/128), the last
+ *     block may be shorter).
+ *   Per block: e = the smallest integer with 448 * 2^e >= max|x| (0 for an all-zero block),
+ *     clamped to [-126, 127]; UE8M0 byte e + 127; code = x * 2^-e rounded to the nearest
+ *     E4M3 value (ties to even, sign kept).
+ *   q [rows][ld_q] uint8 E4M3 codes; sf int16 [ceil(cols/256)][ld_sf] SF words (layout
+ *     above, MN = scale rows; words of rows >= MN and the high byte past an odd block count
+ *     are 0) — what gemm_fp8_nt takes as sfa (block_rows 1) or sfb (block_rows 128,
+ *     sfb_gran_n = 128).
+ *   cols: positive multiple of 128.  ld_x >= cols, ld_q >= cols, ld_sf >= scale rows; x, q,
+ *   sf 16-byte aligned, ld_x * element size, ld_q and ld_sf * 2 multiples of 16 bytes.  The
+ *   buffers must not overlap.  All memory is the caller's; nothing is allocated.
+ */
+int quantize_fp8_ue8m0(const void* x, int in_kind, int rows, int cols, int64_t ld_x, int block_rows,
+                       void* q, int64_t ld_q, void* sf, int64_t ld_sf, void* stream);
+
+/*
  * gemm_fp8_nt_noalloc — the FP8 block-scaled GEMM of gemm_fp8_nt for callers that cannot
  * allocate device memory.  (The pages have no counterpart; this is a deployment variant.)
  *

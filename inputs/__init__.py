@@ -13,6 +13,7 @@ from .synth import (  # noqa: F401
     quantize_e4m3_blocks,
     quantize_e2m1_blocks,
     bf16_operand,
+    normal_matrix,
     dense_fp8_problem,
     dense_fp4_problem,
     dense_bf16_problem,

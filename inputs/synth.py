@@ -110,6 +110,16 @@ def _normal_rows(rng: np.random.Generator, rows: int, k: int):
         yield r0, rng.standard_normal((n, k), dtype=np.float32)
 
 
+def normal_matrix(rows: int, k: int, seed: int, bf16: bool = False) -> np.ndarray:
+    """Unquantised operand for the quantiser: fp32 N(0,1) [rows, k] from ``default_rng(seed)``
+    (the same draw the quantised operands start from), or its bf16 rounding as uint16 bits."""
+    rng = np.random.default_rng(seed)
+    x = np.empty((rows, k), np.float32)
+    for r0, chunk in _normal_rows(rng, rows, k):
+        x[r0:r0 + chunk.shape[0]] = chunk
+    return bf16_operand(x) if bf16 else x
+
+
 def _fp8_operand(rows: int, k: int, seed: int, block_rows: int):
     rng = np.random.default_rng(seed)
     codes = np.empty((rows, k), np.uint8)

@@ -77,6 +77,17 @@ def test_rejects_bad_arguments_without_gpu(lib):
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 4, None) == -3
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 12, None) == -2
     assert lib.transform_sf_ue8m0(good, 1, 64, 8, 8, vp(0x10010), 64, None) == -1
+    # quantiser: kind, block rows, cols not a multiple of 128, ld too small, misaligned ld / pointer
+    qo, so = vp(0x20000), vp(0x30000)
+    assert lib.quantize_fp8_ue8m0(good, 2, 8, 128, 128, 1, qo, 128, so, 8, None) == -1
+    assert lib.quantize_fp8_ue8m0(good, 0, 8, 128, 128, 64, qo, 128, so, 8, None) == -1
+    assert lib.quantize_fp8_ue8m0(None, 0, 8, 128, 128, 1, qo, 128, so, 8, None) == -1
+    assert lib.quantize_fp8_ue8m0(good, 0, 8, 192, 192, 1, qo, 192, so, 8, None) == -3
+    assert lib.quantize_fp8_ue8m0(good, 0, 8, 128, 64, 1, qo, 128, so, 8, None) == -3
+    assert lib.quantize_fp8_ue8m0(good, 0, 16, 128, 128, 1, qo, 128, so, 8, None) == -3  # ld_sf < rows
+    assert lib.quantize_fp8_ue8m0(good, 0, 8, 128, 130, 1, qo, 128, so, 8, None) == -2
+    assert lib.quantize_fp8_ue8m0(good, 0, 8, 128, 128, 1, qo, 136, so, 12, None) == -2
+    assert lib.quantize_fp8_ue8m0(odd, 0, 8, 128, 128, 1, qo, 128, so, 8, None) == -2
 
 
 def test_plan_rejects_bad_arguments_without_gpu(lib):
