@@ -18,5 +18,6 @@ from .synth import (  # noqa: F401
     dense_fp4_problem,
     dense_bf16_problem,
     grouped_fp8_problem,
+    masked_fp8_problem,
     dirichlet_segments,
 )

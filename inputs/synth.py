@@ -20,6 +20,10 @@ Recipe (the one every test, the oracle checks and the bench use):
   integer counts by the largest-remainder rule, each expert segment padded up to
   a multiple of 128 rows.  Padding rows hold zero codes, a unit scale and the
   expert index -1.
+* Masked grouped (decode) layout: every expert owns a slab of max_m rows of A and
+  D; its valid-row count is drawn uniformly from [0, max_m] (``rng.integers``)
+  unless given.  All max_m rows of every slab hold quantised N(0,1) data, so rows
+  past the count carry real-looking values that the GEMM must ignore.
 
 The rounding into E4M3 / E2M1 / bf16 uses ``ml_dtypes`` casts (round to nearest,
 ties to even); the oracle's own decode tables are built independently from the
@@ -211,3 +215,22 @@ def grouped_fp8_problem(groups: int, total_rows: int, n: int, k: int, seed: int 
         b[g], sfb[g] = _fp8_operand(n, k, seed + 2 + g, 128)
     return {"kind": "grouped_fp8", "G": groups, "M": m_total, "N": n, "K": k, "A": a, "sfa": sfa,
             "B": b, "sfb": sfb, "m_indices": m_indices, "counts": counts, "gran_n": 128}
+
+
+def masked_fp8_problem(groups: int, max_m: int, n: int, k: int, seed: int = 0, counts=None):
+    """Masked grouped FP8 problem: A [G, max_m, K] (1x128 scales, [G*max_m, K/128]),
+    B [G, N, K] (128x128 scales), masked_m [G] valid rows per expert."""
+    rng = np.random.default_rng(seed)
+    if counts is None:
+        counts = rng.integers(0, max_m + 1, size=groups)
+    masked_m = np.asarray(counts, dtype=np.int32)
+    if masked_m.shape != (groups,) or masked_m.min() < 0 or masked_m.max() > max_m:
+        raise ValueError("counts must be G values in [0, max_m]")
+    a, sfa = _fp8_operand(groups * max_m, k, seed + 1, 1)
+    b = np.empty((groups, n, k), np.uint8)
+    sfb = np.empty((groups, -(-n // 128), k // 128), np.uint8)
+    for g in range(groups):
+        b[g], sfb[g] = _fp8_operand(n, k, seed + 2 + g, 128)
+    return {"kind": "masked_fp8", "G": groups, "max_m": max_m, "N": n, "K": k,
+            "A": a.reshape(groups, max_m, k), "sfa": sfa, "B": b, "sfb": sfb, "masked_m": masked_m,
+            "gran_n": 128}

@@ -168,6 +168,24 @@ def gemm_grouped_fp8(A, sfa, B, sfb, m_indices, gran_n=128, rows=None, cols=None
     return out
 
 
+def gemm_masked_fp8(A, sfa, B, sfb, masked_m, gran_n=128, rows=None, cols=None) -> np.ndarray:
+    """fp64 D [G*max_m (or rows), N (or cols)] of the masked grouped FP8 GEMM: A [G,max_m,K],
+    sfa [G*max_m, K/128], B [G,N,K], sfb [G, ceil(N/gran_n), K/128], masked_m [G]; rows of
+    expert g at or past masked_m[g] are NaN (not part of the result)."""
+    A, B = _c(A, np.uint8), _c(B, np.uint8)
+    sfa, sfb = _c(sfa, np.uint8), _c(sfb, np.uint8)
+    mm = _c(masked_m, np.int32)
+    (g, max_m, k), n = A.shape, B.shape[1]
+    assert B.shape == (g, n, k) and sfa.shape == (g * max_m, k // 128) and mm.shape == (g,)
+    assert sfb.shape == (g, -(-n // gran_n), k // 128)
+    r, c, nr, nc = _sel(rows, cols, g * max_m, n)
+    out = np.empty((nr, nc))
+    if _load().oracle_gemm_masked_fp8(_p(A), _p(sfa), _p(B), _p(sfb), _p(mm), gran_n, g, max_m, n, k,
+                                      _p(r), nr, _p(c), nc, _p(out)):
+        raise ValueError("gemm_masked_fp8: bad arguments (masked_m outside [0, max_m]?)")
+    return out
+
+
 def quantize_fp8(x, block_rows: int = 1):
     """fp32 (or bf16 bit patterns, uint16) [R, K] -> (E4M3 codes uint8 [R, K],
     biased UE8M0 bytes uint8 [ceil(R/block_rows), K/128]); blocks of block_rows x 128."""

@@ -18,6 +18,11 @@
  *   BF16 D[m,n] = sum_k bf16(A[m,k]) * bf16(B[n,k]).
  *   Grouped (MoE, "Execução de MoE" on the aireiter.com page): row m uses expert
  *        g = m_indices[m] (B := B[g], SFB := SFB[g]); rows with g = -1 are 0.
+ *   Masked grouped (the decode-time MoE layout the crazystack page lists as not
+ *        implemented, "Cobertura de operações e a lacuna declarada no repositório"):
+ *        expert g owns rows [0, max_m) of its own slab of A and D; only rows
+ *        m < masked_m[g] are products, D[g][m] = FP8 formula with B := B[g],
+ *        SFB := SFB[g]; the other rows are not part of the result.
  *   SF packing ("Qué incluye" on the bigchange.ai/es page; "Fatores de escala"
  *        on the crazystack page): each pair of UE8M0 bytes along K goes into one
  *        16-bit word, stored MN-major: out[j*ld + mn] = e[mn][2j] | e[mn][2j+1] << 8.
@@ -264,6 +269,35 @@ int oracle_gemm_grouped_fp8(const uint8_t* A, const uint8_t* sfa, const uint8_t*
                 v = dot_fp8(A + (int64_t)m * K, sfa + (int64_t)m * KB, Bg + (int64_t)n * K,
                             sbg + (int64_t)(n / gran_n) * KB, K);
             }
+            out[(int64_t)i * C + j] = v;
+        }
+    }
+    return 0;
+}
+
+/* Masked grouped FP8: A [G][max_m][K], sfa [G*max_m][K/128], B [G][N][K],
+ * sfb [G][ceil(N/gran_n)][K/128], masked_m [G] with 0 <= masked_m[g] <= max_m.
+ * out [G][max_m][N]: the products for m < masked_m[g]; rows past masked_m[g] are
+ * set to NAN (not part of the result).  rows (NULL = all) selects rows of the
+ * flattened [G*max_m] row index; cols selects columns. */
+int oracle_gemm_masked_fp8(const uint8_t* A, const uint8_t* sfa, const uint8_t* B, const uint8_t* sfb,
+                           const int32_t* masked_m, int gran_n, int G, int max_m, int N, int K,
+                           const int32_t* rows, int nrows, const int32_t* cols, int ncols, double* out) {
+    if (K % 128 || gran_n < 1 || G < 1 || max_m < 0 || N < 0) return -1;
+    for (int g = 0; g < G; ++g)
+        if (masked_m[g] < 0 || masked_m[g] > max_m) return -1;
+    build_tables();
+    int R = rows ? nrows : G * max_m, C = cols ? ncols : N, KB = K / 128, NB = (N + gran_n - 1) / gran_n;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < R; ++i) {
+        int r = rows ? rows[i] : i;
+        int g = r / max_m, m = r % max_m;
+        for (int j = 0; j < C; ++j) {
+            int n = cols ? cols[j] : j;
+            double v = NAN;
+            if (m < masked_m[g])
+                v = dot_fp8(A + (int64_t)r * K, sfa + (int64_t)r * KB, B + ((int64_t)g * N + n) * K,
+                            sfb + ((int64_t)g * NB + n / gran_n) * KB, K);
             out[(int64_t)i * C + j] = v;
         }
     }

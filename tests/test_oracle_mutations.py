@@ -35,6 +35,8 @@ MUTANTS = {
                                    "for (int r = r0; r < r0 + 1; ++r)\n                for (int c = kb * 128; c < kb * 128 + 128; ++c) {\n                    double a"),
     "quant_no_clamp": ("if (ex < -126) ex = -126;", "if (ex < -127) ex = -127;"),
     "quant_subnormal_step": ("ldexp(1.0, -9) : ldexp(1.0, E - 3);", "ldexp(1.0, -10) : ldexp(1.0, E - 3);"),
+    "masked_expert0_weights": ("B + ((int64_t)g * N + n) * K,", "B + ((int64_t)0 * N + n) * K,"),
+    "masked_off_by_one": ("if (m < masked_m[g])", "if (m <= masked_m[g] && m < max_m)"),
     "bf16_sign": ("acc += decode_bf16(A[(int64_t)m * K + k]) * decode_bf16(B[(int64_t)n * K + k]);",
                   "acc -= decode_bf16(A[(int64_t)m * K + k]) * decode_bf16(B[(int64_t)n * K + k]);"),
 }

@@ -411,3 +411,48 @@ def test_quantize_agrees_with_the_input_generator(orc, block_rows):
     q, e = orc.quantize_fp8(x, block_rows)
     q2, e2 = inputs.quantize_e4m3_blocks(x, block_rows)
     assert np.array_equal(q, q2) and np.array_equal(e, e2)
+
+
+# ---------------------------------------------------------------- masked grouped
+
+def test_masked_equals_dense_per_expert(orc):
+    import inputs
+
+    p = inputs.masked_fp8_problem(4, 128, 96, 256, seed=5, counts=[0, 128, 37, 1])
+    got = orc.gemm_masked_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["masked_m"]).reshape(4, 128, 96)
+    for g, c in enumerate(p["masked_m"]):
+        if c:
+            ref = orc.gemm_fp8(p["A"][g, :c], p["sfa"][g * 128:g * 128 + c], p["B"][g], p["sfb"][g])
+            assert np.array_equal(got[g, :c], ref)
+        assert np.isnan(got[g, c:]).all()
+
+
+def test_masked_exact_vs_fraction(orc):
+    rng = np.random.default_rng(8)
+    G, max_m, n, k = 2, 3, 2, 128
+    codes = _all_e4m3()
+    ok = np.flatnonzero(~np.isnan(codes)).astype(np.uint8)
+    A = rng.choice(ok, size=(G, max_m, k)).astype(np.uint8)
+    B = rng.choice(ok, size=(G, n, k)).astype(np.uint8)
+    sfa = rng.integers(120, 134, size=(G * max_m, 1)).astype(np.uint8)
+    sfb = rng.integers(120, 134, size=(G, 1, 1)).astype(np.uint8)
+    mm = np.array([2, 3], np.int32)
+    got = orc.gemm_masked_fp8(A, sfa, B, sfb, mm)
+    for g in range(G):
+        for m in range(max_m):
+            for j in range(n):
+                v = got[g * max_m + m, j]
+                if m >= mm[g]:
+                    assert np.isnan(v)
+                    continue
+                s = sum(Fraction(codes[A[g, m, q]]) * Fraction(codes[B[g, j, q]]) for q in range(k))
+                ref = s * Fraction(2) ** (int(sfa[g * max_m + m, 0]) - 127) * Fraction(2) ** (int(sfb[g, 0, 0]) - 127)
+                assert Fraction(v) == ref
+
+
+def test_masked_rejects_counts_out_of_range(orc):
+    import inputs
+
+    p = inputs.masked_fp8_problem(2, 128, 64, 128, seed=1, counts=[3, 4])
+    with pytest.raises(ValueError):
+        orc.gemm_masked_fp8(p["A"], p["sfa"], p["B"], p["sfb"], np.array([3, 129], np.int32))
