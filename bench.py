@@ -9,7 +9,8 @@ The L2 is flushed (1 GiB write) before every timed step; the flush is outside th
 The same line also reports, each measured the same way (W warm-up, flushed L2, CUDA
 events on the launching stream): BF16 dense at the same shape, FP4 E2M1 at the same
 shape, the M-grouped FP8 MoE workload (32 experts, 32768 rows, N=4096, K=7168), the FP8
-M sweep {128, 1024, 4096} at N=K=7168, the scale transform alone (GB/s), and the FP8
+M sweep {128, 1024, 4096} at N=K=7168, the masked grouped (decode) layout (32 experts x 256
+rows, N=4096, K=7168), the scale transform alone (GB/s), and the FP8
 quantiser that produces the GEMM's operands (fp32 A in 1x128 blocks, bf16 B in 128x128
 blocks, GB/s).
 
@@ -66,8 +67,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only-headline", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "sf_transform", "quantize_act",
-                                          "quantize_wgt"],
+    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "masked", "sf_transform",
+                                          "quantize_act", "quantize_wgt"],
                     help="launch only this kernel (warm-up + steps launches, no timing) for an ncu capture")
     return ap.parse_args()
 
@@ -426,6 +427,32 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
                         "traffic": profiled_traffic("gemm_grouped_fp8_32x32768x4096x7168.md")})
     out[k] = v
 
+    # masked grouped (decode-time MoE): 32 experts, slabs of 256 rows, counts uniform in [0, 256]
+    # drawn from the seed, N = 4096, K = 7168; every expert with rows streams its whole B
+    pm = inputs.masked_fp8_problem(32, 256, 4096, 7168, seed=12)
+    dm = {key: torch.from_numpy(pm[key]).cuda() for key in ("A", "sfa", "B", "masked_m")}
+    sfa_m = ops.transform_sf_ue8m0(dm["sfa"])
+    sfb_m = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(pm["sfb"][e]).cuda()) for e in range(32)])
+    Dm = torch.empty((32, 256, 4096), dtype=torch.bfloat16, device="cuda")
+
+    def f_m(ev):
+        if ev is not None:
+            ev[0].record()
+        ops.m_grouped_gemm_fp8_nt_masked(dm["A"], sfa_m, dm["B"], sfb_m, dm["masked_m"], Dm)
+        if ev is not None:
+            ev[1].record()
+
+    ms = float(timer.run(f_m, args.warmup, reps)[:, 0].mean())
+    rows_valid = int(pm["masked_m"].sum())
+    experts_used = int((pm["masked_m"] > 0).sum())
+    moved = experts_used * 4096 * 7168 + rows_valid * (7168 + 2 * 4096)  # B of used experts, A and D rows
+    k, v = _gemm_entry("masked_fp8_32x256x4096x7168", gemm_flops(rows_valid, 4096, 7168), ms, bf16_peak * 2,
+                       {"rows_valid": rows_valid, "gbs_min_bytes": round(moved / (ms * 1e-3) / 1e9, 1),
+                        "hbm_frac_min_bytes": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "traffic": profiled_traffic("gemm_masked_fp8_32x256x4096x7168.md")})
+    out[k] = v
+    del pm, dm, sfa_m, sfb_m, Dm
+
     # scale transform alone: config-3 SFA (fp32 scales [M_total, 56]) -> int16 words
     s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()
     w = torch.empty((28, ops.sf_ld(g["M"])), dtype=torch.int16, device="cuda")
@@ -558,6 +585,13 @@ def run_profile(args):
         sb = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(g["sfb"][e]).cuda()) for e in range(32)])
         D = torch.empty((g["M"], 4096), dtype=torch.bfloat16, device="cuda")
         fn = lambda: ops.m_grouped_gemm_fp8_nt_contiguous(dg["A"], sa, dg["B"], sb, dg["m_indices"], D)  # noqa
+    elif args.profile == "masked":
+        pm = inputs.masked_fp8_problem(32, 256, 4096, 7168, seed=12)
+        dm = {key: torch.from_numpy(pm[key]).cuda() for key in ("A", "sfa", "B", "masked_m")}
+        sa = ops.transform_sf_ue8m0(dm["sfa"])
+        sb = torch.stack([ops.transform_sf_ue8m0(torch.from_numpy(pm["sfb"][e]).cuda()) for e in range(32)])
+        D = torch.empty((32, 256, 4096), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.m_grouped_gemm_fp8_nt_masked(dm["A"], sa, dm["B"], sb, dm["masked_m"], D)  # noqa: E731
     elif args.profile in ("quantize_act", "quantize_wgt"):
         act = args.profile == "quantize_act"
         xh = inputs.normal_matrix(M if act else N, K, seed=60 + (M if act else N), bf16=not act)

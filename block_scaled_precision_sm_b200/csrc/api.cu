@@ -238,6 +238,7 @@ using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
 using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
 using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
+using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 // M <= 128 with few 224-wide tiles: 64-wide tiles put ~3.5x more SMs on the (B-bandwidth-bound)
 // problem, and their 24 KB stages allow a deeper ring.
 using CfgBF16N = GemmCfg<Kind::BF16, 64, 8, false, false>;
@@ -635,6 +636,35 @@ int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void*
     a.m_indices = m_indices, a.G = G;
     a.sfb_gran = sfb_gran_n;
     return launch_gemm<CfgGrouped>(o, a, *ctx, static_cast<cudaStream_t>(stream));
+}
+
+int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, const void* sfb, void* D,
+                                 const int32_t* masked_m, int G, int max_m, int N, int K, int64_t ld_sfa,
+                                 int64_t ld_sfb, int sfb_gran_n, void* stream) {
+    if (!A || !sfa || !B || !sfb || !D || !masked_m || G < 1 || max_m <= 0 || N <= 0 || K <= 0) return BSP_ERR_ARG;
+    if (sfb_gran_n != 1 && sfb_gran_n != 128) return BSP_ERR_ARG;
+    if (G > CfgMasked::MAX_MASKED_G) return BSP_ERR_UNSUPPORTED;
+    if (K % 128 || max_m % 128) return BSP_ERR_SHAPE;
+    if ((int64_t)G * max_m > 0x7fffffff) return BSP_ERR_UNSUPPORTED;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned16(sfb)) return BSP_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(masked_m) & 3u) != 0) return BSP_ERR_ALIGN;
+    if ((N * 2) % 16) return BSP_ERR_ALIGN;  // rows of D are N bf16 long
+    const int kb = K / 128, words = (kb + 1) / 2;
+    const int mn_b = (N + sfb_gran_n - 1) / sfb_gran_n;
+    const int M = G * max_m;
+    BSP_TRY(check_ld(ld_sfa, M, 2));
+    BSP_TRY(check_ld(ld_sfb, mn_b, 2));
+    DeviceCtx* ctx;
+    BSP_TRY(ensure_ctx(&ctx));
+    Operands o{A, B, sfa, sfb, K, K, ld_sfa, ld_sfb, mn_b, words};
+    o.groups = G;
+    GemmArgs a{};
+    a.M = M, a.N = N, a.K = K;
+    a.D = static_cast<__nv_bfloat16*>(D), a.ldd = N;
+    a.G = G;
+    a.masked_m = masked_m, a.max_m = max_m;
+    a.sfb_gran = sfb_gran_n;
+    return launch_gemm<CfgMasked>(o, a, *ctx, static_cast<cudaStream_t>(stream));
 }
 
 int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in, void* sf_out, int64_t ld_out,

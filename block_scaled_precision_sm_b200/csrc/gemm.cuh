@@ -72,9 +72,11 @@ struct GemmArgs {
     int num_work;  // full_tiles + (num_tiles - full_tiles) * splits
     float* ws;
     int* tail_count;
+    const int32_t* masked_m;  // masked layout: valid rows per expert [G]
+    int max_m;                // masked layout: rows per expert slab
 };
 
-template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2>
+template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
     static constexpr bool PAIR = PAIR_;
@@ -85,6 +87,11 @@ struct GemmCfg {
     static constexpr int BN_CTA = BN / CTAS;    // B rows loaded per CTA
     static constexpr int STAGES = STAGES_;
     static constexpr bool GROUPED = GROUPED_;
+    // masked grouped layout: expert g owns rows [g*max_m, (g+1)*max_m) of A and D, of which
+    // the first masked_m[g] (a device array) are computed; the tile list is built on the device
+    static constexpr bool MASKED = MASKED_;
+    static constexpr int MAX_MASKED_G = 1024;
+    static_assert(!MASKED || (GROUPED && !PAIR_), "masked layout: single-CTA grouped configs only");
     static constexpr bool SCALED = KIND != Kind::BF16;
     // TMEM accumulators: two let the next tile's MMAs run under this tile's epilogue; with one,
     // the epilogue reads the whole accumulator into registers first and releases it at once
@@ -127,7 +134,10 @@ struct GemmCfg {
     static constexpr int NUM_BARS = 2 * STAGES + 5;
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+    // masked layout: valid m-blocks before each expert [G + 1] and the clamped counts [G]
+    static constexpr int OFF_MASK = OFF_MISC + 16;
+    static constexpr int MASK_BYTES = MASKED ? (2 * MAX_MASKED_G + 1) * 4 : 0;
+    static constexpr int SMEM_BYTES = OFF_MASK + MASK_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     // a K slice of a split tile is a worker's last work item, so its epilogue stages the
     // fp32 partial sums (BM x BN) in the then idle A/B stage buffers
@@ -154,6 +164,25 @@ __device__ __forceinline__ Work work_of(const GemmArgs& a, int w, int period) {
     const int groups = (a.num_kb + period - 1) / period;
     const int g0 = j * groups / a.splits, g1 = (j + 1) * groups / a.splits;
     return Work{a.full_tiles + tail, g0 * period, min(g1 * period, a.num_kb), tail, j};
+}
+
+// Masked layout: work item w is n-block w % n_blocks of the (w / n_blocks)-th valid 128-row
+// block, counting the valid blocks of expert 0 first; mprefix[g] holds the valid blocks before
+// expert g.  Returns the block's first row (in the flattened [G * max_m] rows) and its expert.
+__device__ __forceinline__ void masked_tile(const GemmArgs& a, const int* mprefix, int w, int* m0, int* n_blk,
+                                            int* g) {
+    const int mbi = w / a.n_blocks;
+    *n_blk = w - mbi * a.n_blocks;
+    int lo = 0, hi = a.G - 1;  // the expert whose blocks include mbi: smallest g with mprefix[g + 1] > mbi
+    while (lo < hi) {
+        const int mid = (lo + hi) / 2;
+        if (mprefix[mid + 1] > mbi)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    *g = lo;
+    *m0 = lo * a.max_m + (mbi - mprefix[lo]) * 128;
 }
 
 __device__ __forceinline__ Tile tile_of(const GemmArgs& a, int t) {
@@ -271,6 +300,38 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tmem_relinquish();
         }
     }
+    int* mprefix = reinterpret_cast<int*>(smem + C::OFF_MASK);
+    int* mcount = mprefix + C::MAX_MASKED_G + 1;
+    if constexpr (C::MASKED) {
+        // the tile list of the masked layout: valid 128-row blocks per expert, prefix-summed by
+        // one warp (each lane a run of experts, then an exclusive scan over the lanes)
+        if (warp == 2) {
+            const int G = args.G, per = (G + 31) / 32;
+            const int i0 = min(G, (int)lane * per), i1 = min(G, i0 + per);
+            int local = 0;
+            for (int i = i0; i < i1; ++i) {
+                int c = __ldg(args.masked_m + i);
+                if (c < 0 || c > args.max_m) {
+                    latch_status(args.status, kStatusDeviceCheck);
+                    c = c < 0 ? 0 : args.max_m;
+                }
+                mcount[i] = c;
+                local += (c + C::BM - 1) / C::BM;
+            }
+            int incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if ((int)lane >= o) incl += v;
+            }
+            int run = incl - local;
+            for (int i = i0; i < i1; ++i) {
+                mprefix[i] = run;
+                run += (mcount[i] + C::BM - 1) / C::BM;
+            }
+            if (lane == 31) mprefix[G] = incl;
+        }
+    }
     tc_fence_before();
     if constexpr (C::PAIR)
         cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
@@ -278,6 +339,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
+    const int num_work = C::MASKED ? mprefix[args.G] * args.n_blocks : args.num_work;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -285,20 +347,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             bool prior_done = false;  // the scale chunks come from the kernel launched before
-            for (int w = worker; w < args.num_work && ok; w += workers) {
-                const Work wk = work_of(args, w, C::SF_PERIOD);
-                const Tile tl = tile_of(args, wk.tile);
-                const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
-                const int n0 = tl.n_blk * C::BN;
-                const int nb0 = n0 + (int)rank * C::BN_CTA;
-                int g = 0;
-                if constexpr (C::GROUPED) {
-                    g = __ldg(args.m_indices + m0);
-                    if (g < 0 || g >= args.G) {
-                        latch_status(args.status, kStatusDeviceCheck);
-                        g = 0;
+            for (int w = worker; w < num_work && ok; w += workers) {
+                Work wk{0, 0, args.num_kb, -1, 0};
+                int m0, n_blk, g = 0;
+                if constexpr (C::MASKED) {
+                    masked_tile(args, mprefix, w, &m0, &n_blk, &g);
+                } else {
+                    wk = work_of(args, w, C::SF_PERIOD);
+                    const Tile tl = tile_of(args, wk.tile);
+                    m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
+                    n_blk = tl.n_blk;
+                    if constexpr (C::GROUPED) {
+                        g = __ldg(args.m_indices + m0);
+                        if (g < 0 || g >= args.G) {
+                            latch_status(args.status, kStatusDeviceCheck);
+                            g = 0;
+                        }
                     }
                 }
+                const int n0 = n_blk * C::BN;
+                const int nb0 = n0 + (int)rank * C::BN_CTA;
                 for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
@@ -327,7 +395,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (sf_here) {
                             // scale chunks: this CTA's A rows, all BN B rows of the tile
                             tma_load_3d_pair(sf, &tm_sfa, lead_full, 0, m0 / C::BM, q);
-                            tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, tl.n_blk, q);
+                            tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q);
                         }
                     } else {
                         tma_load_2d(sa, &tm_a, &full[s], kx, m0);
@@ -338,9 +406,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (sf_here) {
                             tma_load_3d(sf, &tm_sfa, &full[s], 0, m0 / C::BM, q);
                             if constexpr (C::GROUPED)
-                                tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, tl.n_blk, q, g);
+                                tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q, g);
                             else
-                                tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, tl.n_blk, q);
+                                tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q);
                         }
                     }
                 }
@@ -358,8 +426,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) {
             uint32_t it = 0, lt = 0, git = 0;
             bool ok = true;
-            for (int w = worker; w < args.num_work && ok; w += workers, ++lt) {
-                const Work wk = work_of(args, w, C::SF_PERIOD);
+            for (int w = worker; w < num_work && ok; w += workers, ++lt) {
+                const Work wk = C::MASKED ? Work{0, 0, args.num_kb, -1, 0} : work_of(args, w, C::SF_PERIOD);
                 const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
                 const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
                 if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
@@ -465,18 +533,32 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t quarter = warp % 4;  // TMEM lanes this warp may read
         uint8_t* epi = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BLOCK;
         uint32_t lt = 0, nblk = 0;
-        for (int w = worker; w < args.num_work; w += workers, ++lt) {
-            const Work wk = work_of(args, w, C::SF_PERIOD);
-            const Tile tl = tile_of(args, wk.tile);
-            const int m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
-            const int n0 = tl.n_blk * C::BN;
+        for (int w = worker; w < num_work; w += workers, ++lt) {
+            Work wk{0, 0, args.num_kb, -1, 0};
+            int m0, n_blk, g = 0;
+            if constexpr (C::MASKED) {
+                masked_tile(args, mprefix, w, &m0, &n_blk, &g);
+            } else {
+                wk = work_of(args, w, C::SF_PERIOD);
+                const Tile tl = tile_of(args, wk.tile);
+                m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
+                n_blk = tl.n_blk;
+            }
+            const int n0 = n_blk * C::BN;
             const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
             const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
             if (!warp_wait(&tmem_full[buf], aph, args, abort_flag)) break;
             tc_fence_after();
             const int row = m0 + (int)(quarter * 32 + lane);
             bool zero_row = false;
-            if constexpr (C::GROUPED) {
+            // masked layout: only rows below the expert's count are written; a warp whose 32
+            // rows are all valid stores through TMA, one with some invalid rows row by row
+            bool row_valid = true, all_valid = true;
+            if constexpr (C::MASKED) {
+                row_valid = row - g * args.max_m < mcount[g];
+                all_valid = __all_sync(0xffffffffu, row_valid);
+            }
+            if constexpr (C::GROUPED && !C::MASKED) {
                 if (row < args.M) {
                     const int g0 = __ldg(args.m_indices + m0);
                     const int gi = __ldg(args.m_indices + row);
@@ -502,6 +584,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // one 32 x 32 block (16 packed bf16 pairs per lane) through the swizzled staging
             // buffer to D
             const auto store_block = [&](int c, const uint32_t* w16) {
+                if (!all_valid) {
+                    if (row_valid) {
+                        __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n0 + c * 32;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (n0 + c * 32 + 8 * q + 8 <= args.N)
+                                *reinterpret_cast<uint4*>(dst + 8 * q) =
+                                    make_uint4(w16[4 * q], w16[4 * q + 1], w16[4 * q + 2], w16[4 * q + 3]);
+                    }
+                    return;
+                }
                 // the store issued from this buffer two blocks ago has finished reading it
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();

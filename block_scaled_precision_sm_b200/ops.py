@@ -163,6 +163,39 @@ def m_grouped_gemm_fp8_nt_contiguous(A, sfa, B, sfb, m_indices, D=None, sfb_gran
     return D
 
 
+def m_grouped_gemm_fp8_nt_masked(A, sfa, B, sfb, masked_m, D=None, sfb_gran_n: int = 128,
+                                 stream=None) -> torch.Tensor:
+    """Masked grouped FP8 GEMM: A [G, max_m, K], B [G, N, K], masked_m int32 [G] on the device;
+    D [G, max_m, N] gets rows m < masked_m[g] of every expert (the other rows are not written)."""
+    A8 = _bytes_u8(A)
+    B8 = _bytes_u8(B)
+    if A8.dim() != 3 or B8.dim() != 3 or not A8.is_contiguous() or not B8.is_contiguous():
+        raise ValueError("A [G, max_m, K] and B [G, N, K] must be contiguous")
+    if masked_m.dtype != torch.int32 or not masked_m.is_contiguous() or not masked_m.is_cuda:
+        raise ValueError("masked_m must be a contiguous int32 device tensor")
+    (g, max_m, k), n = A8.shape, B8.shape[1]
+    if B8.shape[0] != g or B8.shape[2] != k or masked_m.numel() != g:
+        raise ValueError("A, B and masked_m disagree on G or K")
+    kb = k // 128
+    sfa = packed_sf(sfa.reshape(g * max_m, -1) if sfa.dim() == 3 and sfa.dtype != torch.int16 else sfa,
+                    g * max_m, kb, stream)
+    mn_b = -(-n // sfb_gran_n)
+    if sfb.dim() == 3 and sfb.dtype == torch.int16:
+        if sfb.shape[0] != g or sfb.shape[1] != (kb + 1) // 2 or sfb.shape[2] < mn_b or not sfb.is_contiguous():
+            raise ValueError("packed sfb must be contiguous int16 [G, words, ld]")
+    else:
+        if sfb.dim() != 3 or tuple(sfb.shape) != (g, mn_b, kb):
+            raise ValueError(f"sfb must be packed int16 [G, words, ld] or [{g}, {mn_b}, {kb}]")
+        sfb = torch.stack([transform_sf_ue8m0(sfb[i], stream=stream) for i in range(g)])
+    if D is None:
+        D = torch.empty((g, max_m, n), dtype=torch.bfloat16, device=A8.device)
+    if D.dtype != torch.bfloat16 or tuple(D.shape) != (g, max_m, n) or not D.is_contiguous():
+        raise ValueError("D must be contiguous bf16 [G, max_m, N]")
+    _lib.call("m_grouped_gemm_fp8_nt_masked", _ptr(A8), _ptr(sfa), _ptr(B8), _ptr(sfb), _ptr(D),
+              _ptr(masked_m), g, max_m, n, k, sfa.stride(0), sfb.stride(1), sfb_gran_n, _stream(stream))
+    return D
+
+
 def device_status(stream=None) -> int:
     """Synchronise and return (and clear) the status word latched by the kernels."""
     return _lib.load().bsp_get_device_status(_stream(stream))

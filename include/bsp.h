@@ -116,6 +116,27 @@ int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void*
                                      void* stream);
 
 /*
+ * m_grouped_gemm_fp8_nt_masked — M-grouped FP8 GEMM in the masked (decode-time) layout,
+ * which the pages list as not yet implemented in their release ("DeepGEMM-Ascend cobre
+ * quantas operações no Ascend 950?", section "Cobertura de operações e a lacuna declarada no
+ * repositório").  Every expert g owns a slab of max_m rows; only the first masked_m[g] rows of
+ * the slab are products, the count being read on the device (so a CUDA graph can be captured
+ * before the routing that produces it is known):
+ *   D[g][m][n] = FP8 formula above with B := B[g], SFB := SFB[g]   for m < masked_m[g];
+ *   rows m >= masked_m[g] of D are not written (they keep whatever they held).
+ *   A [G][max_m][K] E4M3; sfa SF words for MN = G*max_m (row g*max_m + m), ld_sfa.
+ *   B [G][N][K] E4M3; sfb [G][ceil(KB/2)][ld_sfb] SF words per expert, MN = ceil(N/sfb_gran_n).
+ *   D [G][max_m][N] bf16.  masked_m int32 [G] in device memory, values in [0, max_m]; a value
+ *   outside latches BSP_ERR_DEVICE_CHECK and is clamped into the range.
+ *   1 <= G <= 1024; max_m a positive multiple of 128; K a positive multiple of 128; N*2 a
+ *   multiple of 16 bytes.  The work is split by the device-side counts: tiles of rows past
+ *   masked_m[g] are neither loaded nor computed.
+ */
+int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, const void* sfb, void* D,
+                                 const int32_t* masked_m, int G, int max_m, int N, int K, int64_t ld_sfa,
+                                 int64_t ld_sfb, int sfb_gran_n, void* stream);
+
+/*
  * transform_sf_ue8m0 — scale factors [mn][kb] (row stride ld_in) into SF words
  * int16 [ceil(kb/2)][ld_out] (layout above).
  *   in_kind 0: fp32 scales, each an exact positive normal power of two; its biased

@@ -77,6 +77,18 @@ def test_rejects_bad_arguments_without_gpu(lib):
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 4, None) == -3
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 12, None) == -2
     assert lib.transform_sf_ue8m0(good, 1, 64, 8, 8, vp(0x10010), 64, None) == -1
+    # masked grouped: max_m not a multiple of 128, G out of range, misaligned counts
+    mm = vp(0x40000)
+    assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, mm, 2, 100, 128, 128, 256, 8, 128,
+                                            None) == -3
+    assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, mm, 0, 128, 128, 128, 256, 8, 128,
+                                            None) == -1
+    assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, mm, 1025, 128, 128, 128, 131200, 8,
+                                            128, None) == -4
+    assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, vp(0x40002), 2, 128, 128, 128, 256, 8,
+                                            128, None) == -2
+    assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, None, 2, 128, 128, 128, 256, 8, 128,
+                                            None) == -1
     # quantiser: kind, block rows, cols not a multiple of 128, ld too small, misaligned ld / pointer
     qo, so = vp(0x20000), vp(0x30000)
     assert lib.quantize_fp8_ue8m0(good, 2, 8, 128, 128, 1, qo, 128, so, 8, None) == -1

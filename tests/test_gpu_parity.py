@@ -321,6 +321,97 @@ def test_grouped_bad_index_is_flagged(ops):
     _status_ok(ops)
 
 
+# ------------------------------------------------------------------ masked grouped
+
+_SENTINEL = 0x3C5A  # a bf16 bit pattern no product of these inputs is likely to round to exactly
+
+
+def _masked(ops, p, D=None):
+    g, max_m, n = p["G"], p["max_m"], p["N"]
+    if D is None:
+        D = torch.full((g, max_m, n), 0, dtype=torch.int16, device="cuda").fill_(_SENTINEL).view(torch.bfloat16)
+    ops.m_grouped_gemm_fp8_nt_masked(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]),
+                                     to_dev(p["masked_m"]), D)
+    return D
+
+
+def _check_masked(orc, p, D, what):
+    g, max_m, n = p["G"], p["max_m"], p["N"]
+    got = bf16_to_f64(D).reshape(g * max_m, n)
+    raw = D.view(torch.int16).cpu().numpy().view(np.uint16).reshape(g * max_m, n)
+    valid = np.concatenate([np.arange(max_m) < c for c in p["masked_m"]])
+    assert (raw[~valid] == _SENTINEL).all(), f"{what}: rows past masked_m were written"
+    if valid.sum() * n >= 1000:
+        ref = orc.gemm_masked_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["masked_m"])
+        check_gemm(got[valid], ref[valid], what)
+
+
+@pytest.mark.parametrize("counts,n,k", [([0, 256, 37, 129], 448, 512), ([1, 128, 255, 64, 0, 200], 1000, 1024)])
+def test_masked(ops, orc, counts, n, k):
+    p = inputs.masked_fp8_problem(len(counts), 256, n, k, seed=len(counts), counts=counts)
+    D = _masked(ops, p)
+    _status_ok(ops)
+    _check_masked(orc, p, D, f"masked {counts}")
+
+
+def test_masked_random_counts(ops, orc):
+    p = inputs.masked_fp8_problem(16, 384, 640, 768, seed=77)
+    D = _masked(ops, p)
+    _status_ok(ops)
+    _check_masked(orc, p, D, "masked random counts")
+
+
+def test_masked_all_empty_writes_nothing(ops):
+    p = inputs.masked_fp8_problem(3, 128, 256, 256, seed=2, counts=[0, 0, 0])
+    D = _masked(ops, p)
+    _status_ok(ops)
+    assert (D.view(torch.int16) == _SENTINEL).all()
+
+
+def test_masked_equals_contiguous_bit_exact(ops):
+    # the same rows through the contiguous layout (each 128-row slab one expert, rows past the
+    # count marked -1) run the same MMAs in the same order: identical bytes on the valid rows
+    counts = [1, 128, 77, 5]
+    p = inputs.masked_fp8_problem(4, 128, 448, 1024, seed=9, counts=counts)
+    Dm = _masked(ops, p)
+    idx = np.concatenate([np.where(np.arange(128) < c, g, -1) for g, c in enumerate(counts)]).astype(np.int32)
+    Dc = ops.m_grouped_gemm_fp8_nt_contiguous(to_dev(p["A"].reshape(512, 1024)), to_dev(p["sfa"]), to_dev(p["B"]),
+                                              to_dev(p["sfb"]), to_dev(idx))
+    _status_ok(ops)
+    valid = torch.from_numpy(idx >= 0).cuda()
+    assert torch.equal(Dm.reshape(512, 448)[valid].view(torch.int16), Dc[valid].view(torch.int16))
+
+
+def test_masked_counts_are_read_on_the_device(ops, orc):
+    # capture once, then change the counts on the device between replays
+    p = inputs.masked_fp8_problem(4, 256, 448, 512, seed=31, counts=[10, 0, 256, 130])
+    dv = {x: to_dev(p[x]) for x in ("A", "sfa", "B", "sfb", "masked_m")}
+    sa = ops.transform_sf_ue8m0(dv["sfa"])
+    sb = torch.stack([ops.transform_sf_ue8m0(dv["sfb"][e]) for e in range(4)])
+    D = torch.empty((4, 256, 448), dtype=torch.bfloat16, device="cuda")
+    ops.m_grouped_gemm_fp8_nt_masked(dv["A"], sa, dv["B"], sb, dv["masked_m"], D)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.m_grouped_gemm_fp8_nt_masked(dv["A"], sa, dv["B"], sb, dv["masked_m"], D)
+    for counts in ([10, 0, 256, 130], [256, 3, 0, 129]):
+        dv["masked_m"].copy_(torch.tensor(counts, dtype=torch.int32))
+        D.view(torch.int16).fill_(_SENTINEL)
+        g.replay()
+        torch.cuda.synchronize()
+        _status_ok(ops)
+        q = dict(p, masked_m=np.array(counts, np.int32))
+        _check_masked(orc, q, D, f"replay {counts}")
+
+
+def test_masked_bad_count_is_flagged(ops):
+    p = inputs.masked_fp8_problem(2, 128, 256, 256, seed=4, counts=[5, 7])
+    q = dict(p, masked_m=np.array([5, 300], np.int32))  # 300 > max_m: clamped to 128 and flagged
+    _masked(ops, q)
+    assert ops.device_status() == -7
+    _status_ok(ops)
+
+
 # ------------------------------------------------------------------ failure detection
 
 def test_wait_timeout_is_reported_and_context_survives(ops, orc):
