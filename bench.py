@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--only-headline", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--profile", choices=["fp8", "bf16", "fp4", "grouped", "masked", "sf_transform",
+    ap.add_argument("--profile", choices=["fp8", "fp8_m128", "bf16", "fp4", "grouped", "masked", "sf_transform",
                                           "quantize_act", "quantize_wgt"],
                     help="launch only this kernel (warm-up + steps launches, no timing) for an ncu capture")
     return ap.parse_args()
@@ -565,6 +565,11 @@ def run_profile(args):
         p, dv = fp8_device_problem(torch, M, N, K, seed=100)
         sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
         D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # noqa: E731
+    elif args.profile == "fp8_m128":
+        p, dv = fp8_device_problem(torch, 128, 7168, 7168, seed=30 + 128)
+        sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
+        D = torch.empty((128, 7168), dtype=torch.bfloat16, device="cuda")
         fn = lambda: ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # noqa: E731
     elif args.profile == "bf16":
         p = inputs.dense_bf16_problem(M, N, K, seed=2)

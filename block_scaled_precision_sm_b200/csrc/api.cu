@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "bsp.h"
 #include "gemm.cuh"
@@ -138,8 +139,8 @@ int max_workers_of(const DeviceCtx& ctx, int* out) {
 
 // Tail plan: how many whole tiles, and into how many K slices the rest is cut.  The tiles
 // left over after the last full wave of workers are split when at least two slices of
-// eight or more K steps fit per tile, up to 16 slices, so that the last wave keeps most
-// workers busy instead of a few.
+// eight or more K steps fit per tile, up to 16 slices (a power of two), so that the last
+// wave keeps most workers busy instead of a few.
 struct TailPlan {
     int tiles, full_tiles, splits, tail_tiles, num_work;
 };
@@ -153,6 +154,7 @@ TailPlan plan_tail(int tiles, int num_kb, int period, int workers, bool allow) {
     s = s < 16 ? s : 16;
     s = s < groups ? s : groups;
     while (s >= 2 && num_kb / s < 8) --s;
+    while (s & (s - 1)) --s;  // a power of two: every slice then sums 32/S rows of each warp
     if (s < 2) return p;
     p.full_tiles = tiles - rem;
     p.splits = s;
@@ -235,23 +237,28 @@ using CfgBF16P256 = GemmCfg<Kind::BF16, 256, 6, false, true, 1>;
 using CfgFP8P256 = GemmCfg<Kind::FP8, 256, 6, false, true, 1>;
 using CfgFP4P256 = GemmCfg<Kind::FP4, 256, 5, false, true, 1>;
 using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
-using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
+using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;  // constants only (FP8 M <= 128 runs swapped)
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
 using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 // M <= 128 with few 224-wide tiles: 64-wide tiles put ~3.5x more SMs on the (B-bandwidth-bound)
 // problem, and their 24 KB stages allow a deeper ring.
 using CfgBF16N = GemmCfg<Kind::BF16, 64, 8, false, false>;
-using CfgFP8N = GemmCfg<Kind::FP8, 64, 8, false, false>;
 using CfgFP4N = GemmCfg<Kind::FP4, 64, 8, false, false>;
+// FP8 with M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair,
+// A's rows across), written transposed.  Per SM and K step: 128 rows of B and 64 of A (24 KB)
+// for 128 x 128 products, against 24 KB for 128 x 64 in the narrow tiles: half the bytes per
+// product, in a kernel whose loads are latency-bound.
+using CfgFP8S = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true>;
 
 // Tile shape by problem shape.  M > 128: CTA pairs, 256 or 224 columns wide, whichever
 // finishes first by a model of the waves (tile time proportional to its MMA work, 224-wide
 // tiles 8% less efficient, a split tail paying for its longest slice plus about four K steps
-// of reduction).  M <= 128: single CTAs, 64 wide when 224-wide tiles would leave most SMs
-// idle.
-enum class Shape { Pair256, Pair224, Wide, Narrow };
-Shape pick_shape(int M, int N, int num_kb, int period, int sms) {
+// of reduction).  M <= 128: FP8 runs transposed on 256 x 128 pair tiles (swap_small_m); the
+// other kinds use single CTAs, 64 wide when 224-wide tiles would leave most SMs idle.
+enum class Shape { Pair256, Pair224, Wide, Narrow, Swap };
+Shape pick_shape(int M, int N, int num_kb, int period, int sms, bool swap_small_m = false) {
+    if (M <= 128 && swap_small_m) return Shape::Swap;
     if (M > 128) {
         const int workers = sms / 2;
         const auto cost = [&](int bn, double eff) {
@@ -280,6 +287,20 @@ struct Operands {
     int groups = 1;   // experts (grouped layout)
 };
 
+// The swapped problem D^T = B A^T: operands, scale tensors and sizes exchanged; B's scale
+// granularity becomes the A-operand's, A's per-row scales the B-operand's.
+void swap_operands(Operands& o, GemmArgs& a) {
+    std::swap(o.A, o.B);
+    std::swap(o.sfa, o.sfb);
+    std::swap(o.lda, o.ldb);
+    std::swap(o.ld_sfa, o.ld_sfb);
+    o.mn_b = a.M;
+    std::swap(a.M, a.N);
+    a.sfa_gran = a.sfb_gran;
+    a.sfb_gran = 1;
+}
+
+
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // Scale chunks of config C: layouts of the A and B chunk tensors and their bytes.
@@ -289,7 +310,8 @@ struct ScaleChunks {
     int64_t a_bytes = 0, b_bytes = 0;
     ScaleChunks(const Operands& o, const GemmArgs& g) {
         const int q = (o.words + 2 * C::UT_WORDS - 1) / (2 * C::UT_WORDS);
-        a = SfLayout{g.M, 1, o.words, o.ld_sfa, 0, C::BM, 1, C::UT_WORDS, (g.M + C::BM - 1) / C::BM, q, 1};
+        a = SfLayout{g.M, g.sfa_gran > 1 ? g.sfa_gran : 1, o.words, o.ld_sfa, 0, C::BM, 1, C::UT_WORDS,
+                     (g.M + C::BM - 1) / C::BM, q, 1};
         const int64_t b_gstride = (int64_t)o.words * o.ld_sfb;
         b = SfLayout{g.N, g.sfb_gran, o.words, o.ld_sfb, b_gstride, C::BN, C::SFB_ATOMS, C::UT_WORDS,
                      (g.N + C::BN - 1) / C::BN, q, o.groups};
@@ -304,7 +326,12 @@ int launch_sf_layout(const void* in_a, const SfLayout& pa, void* out_a, const vo
                      void* out_b, void* zero, int64_t zero_bytes, cudaStream_t stream) {
     const int64_t total = sf_layout_words(pa) + sf_layout_words(pb) + zero_bytes / 16;
     const int64_t blocks = (total + 255) / 256;
-    sf_tmem_layout_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
+    // a grid that is resident at once (grid-stride loop): every CTA reaches the early
+    // launch_dependents right away, so the GEMM after it is launched without waiting
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * 4;
+    sf_tmem_layout_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(
         static_cast<const uint16_t*>(in_a), pa, static_cast<uint32_t*>(out_a), static_cast<const uint16_t*>(in_b),
         pb, static_cast<uint32_t*>(out_b), static_cast<uint4*>(zero), zero_bytes / 16);
     g_launches.fetch_add(1);
@@ -380,6 +407,7 @@ int describe_plan(int M, int N, int K, const DeviceCtx& ctx, int32_t* out) {
     out[3] = p.tail_tiles;
     out[4] = p.num_work;
     out[5] = p.num_work < max_workers ? p.num_work : max_workers;
+    out[6] = 0;
     return BSP_OK;
 }
 
@@ -494,11 +522,15 @@ int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
     a.M = M, a.N = N, a.K = K, a.sfb_gran = sfb_gran_n;
     int sms = 0;
     if (device_facts_noalloc(&sms) != BSP_OK) sms = 148;
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, sms)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, sms, true)) {
         case Shape::Pair256: return ScaleChunks<CfgFP8P256>(o, a).bytes();
         case Shape::Pair224: return ScaleChunks<CfgFP8P224>(o, a).bytes();
-        case Shape::Wide: return ScaleChunks<CfgFP8>(o, a).bytes();
-        default: return ScaleChunks<CfgFP8N>(o, a).bytes();
+        default: {  // Swap: M <= 128
+            Operands os = o;
+            GemmArgs as = a;
+            swap_operands(os, as);
+            return ScaleChunks<CfgFP8S>(os, as).bytes();
+        }
     }
 }
 
@@ -516,11 +548,14 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
     a.M = M, a.N = N, a.K = K;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx.sms)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx.sms, true)) {
         case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, ctx, stream, scratch, scratch_bytes);
         case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, ctx, stream, scratch, scratch_bytes);
-        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, ctx, stream, scratch, scratch_bytes);
-        default: return launch_gemm<CfgFP8N>(o, a, ctx, stream, scratch, scratch_bytes);
+        default: {  // Swap: M <= 128
+            Operands os = o;
+            swap_operands(os, a);
+            return launch_gemm<CfgFP8S>(os, a, ctx, stream, scratch, scratch_bytes);
+        }
     }
 }
 
@@ -577,11 +612,14 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx->sms)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx->sms, true)) {
         case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, *ctx, st);
         case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, *ctx, st);
-        case Shape::Wide: return launch_gemm<CfgFP8>(o, a, *ctx, st);
-        default: return launch_gemm<CfgFP8N>(o, a, *ctx, st);
+        default: {  // Swap: M <= 128
+            Operands os = o;
+            swap_operands(os, a);
+            return launch_gemm<CfgFP8S>(os, a, *ctx, st);
+        }
     }
 }
 
@@ -734,11 +772,14 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                 default: return describe_plan<CfgBF16N>(M, N, K, *ctx, plan);
             }
         case 1:
-            switch (pick_shape(M, N, (K + 127) / 128, CfgFP8::SF_PERIOD, ctx->sms)) {
+            switch (pick_shape(M, N, (K + 127) / 128, CfgFP8::SF_PERIOD, ctx->sms, true)) {
                 case Shape::Pair256: return describe_plan<CfgFP8P256>(M, N, K, *ctx, plan);
                 case Shape::Pair224: return describe_plan<CfgFP8P224>(M, N, K, *ctx, plan);
-                case Shape::Wide: return describe_plan<CfgFP8>(M, N, K, *ctx, plan);
-                default: return describe_plan<CfgFP8N>(M, N, K, *ctx, plan);
+                default: {  // Swap: M <= 128
+                    BSP_TRY(describe_plan<CfgFP8S>(N, M, K, *ctx, plan));
+                    plan[6] = 1;
+                    return BSP_OK;
+                }
             }
         case 2:
             switch (pick_shape(M, N, (K + 255) / 256, CfgFP4::SF_PERIOD, ctx->sms)) {

@@ -58,6 +58,7 @@ struct GemmArgs {
     const int32_t* m_indices;  // grouped layout only
     int G;
     int sfb_gran;              // 1 or 128 (FP8); 1 for FP4
+    int sfa_gran;              // A-operand scale rows per matrix row block (0 or 1: per row)
     int* status;
     unsigned long long timeout_ns;
     // Split tail: the first full_tiles tiles (in raster order) are computed whole, one per
@@ -76,7 +77,8 @@ struct GemmArgs {
     int max_m;                // masked layout: rows per expert slab
 };
 
-template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false>
+template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false,
+          bool TRANS_D_ = false>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
     static constexpr bool PAIR = PAIR_;
@@ -92,6 +94,11 @@ struct GemmCfg {
     static constexpr bool MASKED = MASKED_;
     static constexpr int MAX_MASKED_G = 1024;
     static_assert(!MASKED || (GROUPED && !PAIR_), "masked layout: single-CTA grouped configs only");
+    // the kernel computes D^T = B' A'^T with the caller's operands swapped (A' = B, B' = A) and
+    // writes each accumulator element (row i, column j) to D[j][i]: small-M problems put the
+    // long N dimension on the 256-row pair tiles
+    static constexpr bool TRANS_D = TRANS_D_;
+    static_assert(!TRANS_D || !GROUPED, "transposed output: dense configs only");
     static constexpr bool SCALED = KIND != Kind::BF16;
     // TMEM accumulators: two let the next tile's MMAs run under this tile's epilogue; with one,
     // the epilogue reads the whole accumulator into registers first and releases it at once
@@ -131,7 +138,8 @@ struct GemmCfg {
     static constexpr int EPI_BLOCK = 32 * 32 * 2;
     static constexpr int OFF_EPI = ((OFF_SF + STAGES * SF_STAGE_BYTES + 1023) / 1024) * 1024;
     // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain
-    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail gather
+    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // masked layout: valid m-blocks before each expert [G + 1] and the clamped counts [G]
@@ -257,6 +265,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* tmem_full = empty + C::STAGES;
     uint64_t* tmem_empty = tmem_full + 2;
     uint64_t* drain = tmem_empty + 2;
+    uint64_t* gather = drain + 1;  // [4]: one per epilogue warp
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -278,6 +287,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             mbar_init(&tmem_empty[b], 4 * C::CTAS);
         }
         mbar_init(drain, 1);
+        for (int w = 0; w < 4; ++w) mbar_init(&gather[w], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -532,7 +542,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const uint32_t quarter = warp % 4;  // TMEM lanes this warp may read
         uint8_t* epi = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BLOCK;
-        uint32_t lt = 0, nblk = 0;
+        uint32_t lt = 0, nblk = 0, gather_phase = 0;
         for (int w = worker; w < num_work; w += workers, ++lt) {
             Work wk{0, 0, args.num_kb, -1, 0};
             int m0, n_blk, g = 0;
@@ -584,6 +594,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // one 32 x 32 block (16 packed bf16 pairs per lane) through the swizzled staging
             // buffer to D
             const auto store_block = [&](int c, const uint32_t* w16) {
+                if constexpr (C::TRANS_D) {
+                    // element (row, n0 + 32c + j) goes to D[n0 + 32c + j][row]: for each j the
+                    // warp writes 32 consecutive bf16 of one row of D
+                    if (row < args.M) {
+                        __nv_bfloat16* col = args.D + row;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int d_row = n0 + c * 32 + j;
+                            if (d_row < args.N)
+                                *reinterpret_cast<uint16_t*>(col + (int64_t)d_row * args.ldd) =
+                                    (uint16_t)(w16[j >> 1] >> (16 * (j & 1)));
+                        }
+                    }
+                    return;
+                }
                 if (!all_valid) {
                     if (row_valid) {
                         __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n0 + c * 32;
@@ -667,40 +692,85 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     __threadfence();
                 }
                 if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-                // this slice's share of the 32 rows: sum the slots in order, round, store.  The
-                // (row, slot) pairs are walked four at a time with all their loads in flight.
+                // this slice's share of the 32 rows (32/S of them, S a power of two): gather every
+                // slot's copy of those rows into this warp's (now free) staging area with one
+                // round of bulk copies, then sum the slots in order, round and store
                 const int S = args.splits;
-                const int r0 = wk.slice * 32 / S, r1 = (wk.slice + 1) * 32 / S;
-                const int col = (int)lane * 8;  // 8 columns per lane
-                const int n = n0 + col;
-                const bool col_ok = col < C::BN && n < args.N;
-                const float* base = args.ws + (int64_t)wk.tail * S * slot_stride +
-                                    (int64_t)((int)rank * C::BM + (int)quarter * 32) * C::BN + col;
-                const int pairs = (r1 - r0) * S;
-                float v[8];
-                for (int b = 0; b < pairs; b += 4) {
-                    float4 x[8];
+                const int r0 = wk.slice * (32 / S), nr = 32 / S;
+                const int row_bytes = C::BN * 4;
+                const float* wbase = args.ws + (int64_t)wk.tail * S * slot_stride +
+                                     (int64_t)((int)rank * C::BM + (int)quarter * 32) * C::BN;
+                if (lane == 0) {
+                    fence_proxy_async_global();  // the other slices' stores, acquired above, before these reads
+                    mbar_arrive_expect_tx(&gather[warp - 2], (uint32_t)(nr * S * row_bytes));
+                    for (int i = 0; i < nr; ++i)
+                        for (int j = 0; j < S; ++j)
+                            bulk_load(stage + (i * S + j) * row_bytes, wbase + j * slot_stride + (int64_t)(r0 + i) * C::BN,
+                                      (uint32_t)row_bytes, &gather[warp - 2]);
+                }
+                if (!warp_wait(&gather[warp - 2], gather_phase, args, abort_flag)) break;
+                gather_phase ^= 1u;
+                if constexpr (C::TRANS_D) {
+                    // element (row, n0 + c) goes to D[n0 + c][row]: lane l sums columns 4l .. 4l + 3 of
+                    // the nr rows (16-byte shared loads) and writes nr consecutive bf16 of each of the
+                    // four rows D[n0 + 4l + e]
+                    const int row0 = m0 + (int)quarter * 32 + r0;
+                    const uint32_t sbase = smem_u32(stage);
+                    for (int c4 = (int)lane * 4; c4 < C::BN; c4 += 128) {
+                        float acc[16][4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int pi = b + u, i = r0 + pi / S, j = pi % S;
-                        if (pi < pairs && col_ok && m0 + (int)quarter * 32 + i < args.M) {
-                            const float4* p4 = reinterpret_cast<const float4*>(base + j * slot_stride + (int64_t)i * C::BN);
-                            x[2 * u] = __ldcg(p4);
-                            x[2 * u + 1] = __ldcg(p4 + 1);
+                        for (int i = 0; i < 16; ++i) {
+                            acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+                            if (i < nr)
+                                for (int j = 0; j < S; ++j) {
+                                    const float4 x = ld_shared_f32x4(sbase + (uint32_t)((i * S + j) * row_bytes + c4 * 4));
+                                    acc[i][0] += x.x, acc[i][1] += x.y, acc[i][2] += x.z, acc[i][3] += x.w;
+                                }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int d_row = n0 + c4 + e;
+                            if (d_row >= args.N) continue;
+                            uint32_t packed[8];
+#pragma unroll
+                            for (int i2 = 0; i2 < 8; ++i2) {
+                                __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(acc[2 * i2][e], acc[2 * i2 + 1][e]));
+                                packed[i2] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
+                            if (row0 + nr <= args.M) {
+                                // nr is 16, 8, 4 or 2 rows: 32, 16, 8 or 4 aligned bytes
+                                if (nr == 16) {
+                                    reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                                    reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                                } else if (nr == 8) {
+                                    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                                } else if (nr == 4) {
+                                    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+                                } else {
+                                    *reinterpret_cast<uint32_t*>(dst) = packed[0];
+                                }
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    if (i < nr && row0 + i < args.M)
+                                        *reinterpret_cast<uint16_t*>(dst + i) = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
+                            }
                         }
                     }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int pi = b + u, i = r0 + pi / S, j = pi % S;
-                        const int row = m0 + (int)quarter * 32 + i;
-                        if (pi >= pairs || !col_ok || row >= args.M) continue;
-                        if (j == 0) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+                } else {
+                    const int col = (int)lane * 8;  // 8 columns per lane
+                    const int n = n0 + col;
+                    for (int i = 0; i < nr; ++i) {
+                        const int row = m0 + (int)quarter * 32 + r0 + i;
+                        if (row >= args.M || col >= C::BN || n >= args.N) continue;
+                        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        for (int j = 0; j < S; ++j) {
+                            const float4* p4 = reinterpret_cast<const float4*>(stage + (i * S + j) * row_bytes + col * 4);
+                            const float4 x0 = p4[0], x1 = p4[1];
+                            v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
+                            v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
                         }
-                        v[0] += x[2 * u].x, v[1] += x[2 * u].y, v[2] += x[2 * u].z, v[3] += x[2 * u].w;
-                        v[4] += x[2 * u + 1].x, v[5] += x[2 * u + 1].y, v[6] += x[2 * u + 1].z, v[7] += x[2 * u + 1].w;
-                        if (j != S - 1) continue;
                         __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
                         if (n + 8 <= args.N) {
                             uint32_t o[4];
@@ -711,7 +781,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             }
                             *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
                         } else {
-                            for (int e = 0; e < 8 && n + e < args.N; ++e) dst[e] = __float2bfloat16_rn(v[e]);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (n + e < args.N) dst[e] = __float2bfloat16_rn(v[e]);
                         }
                     }
                 }

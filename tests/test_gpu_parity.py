@@ -188,6 +188,18 @@ def test_fp4(ops, orc, m, n, k):
     check_gemm(bf16_to_f64(D), orc.gemm_fp4(p["A"], p["sfa"], p["B"], p["sfb"]), f"fp4 {m}x{n}x{k}")
 
 
+# ------------------------------------------------------------------ small M, transposed
+
+@pytest.mark.parametrize("m,n,k,gran", [(128, 7168, 2048, 128), (77, 1000, 1024, 1), (1, 4000, 640, 128),
+                                        (33, 300, 4096, 1), (128, 256, 128, 128)])
+def test_fp8_small_m_runs_transposed(ops, orc, m, n, k, gran):
+    # M <= 128: D^T = B A^T on 256 x 128 pair tiles, written back transposed; ragged N and M,
+    # per-row and 128x128 B scales, split and unsplit plans
+    plan = ops.gemm_plan("fp8", m, n, k)
+    assert plan["transposed"] == 1 and plan["tile_m"] == 256 and plan["tile_n"] == 128, plan
+    _fp8_case(ops, orc, m, n, k, seed=m * 13 + n, gran=gran)
+
+
 # ------------------------------------------------------------------ split last wave
 
 def _run_kind(ops, kind, m, n, k, seed, gran=128, rows=None, cols=None):
