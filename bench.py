@@ -400,7 +400,10 @@ def secondary(torch, ops, timer, args, peaks, peak_kind):
         fl = gemm_flops(m, 7168, 7168)
         sweep[str(m)] = {"tflops": round(fl / (ms * 1e-3) / 1e12, 1), "ms": round(ms, 5),
                          "frac_tensor": round(fl / (ms * 1e-3) / 1e12 / (bf16_peak * 2), 4),
-                         "hbm_gbs_min_bytes": round(bytes_min / (ms * 1e-3) / 1e9, 1)}
+                         "hbm_gbs_min_bytes": round(bytes_min / (ms * 1e-3) / 1e9, 1),
+                         "plan": ops.gemm_plan("fp8", m, 7168, 7168)}
+        if m == 128:
+            sweep[str(m)]["traffic"] = profiled_traffic("gemm_fp8_transposed_128x7168x7168.md")
         del p, dv, sa, sb, Dm
     out["fp8_m_sweep_n7168_k7168"] = sweep
 

@@ -766,8 +766,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (row >= args.M || col >= C::BN || n >= args.N) continue;
                         float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                         for (int j = 0; j < S; ++j) {
-                            const float4* p4 = reinterpret_cast<const float4*>(stage + (i * S + j) * row_bytes + col * 4);
-                            const float4 x0 = p4[0], x1 = p4[1];
+                            const uint32_t a4 = smem_u32(stage) + (uint32_t)((i * S + j) * row_bytes + col * 4);
+                            const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
                             v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
                             v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
                         }
