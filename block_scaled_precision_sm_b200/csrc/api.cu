@@ -236,46 +236,41 @@ using CfgFP4P224 = GemmCfg<Kind::FP4, 224, 6, false, true>;
 using CfgBF16P256 = GemmCfg<Kind::BF16, 256, 6, false, true, 1>;
 using CfgFP8P256 = GemmCfg<Kind::FP8, 256, 6, false, true, 1>;
 using CfgFP4P256 = GemmCfg<Kind::FP4, 256, 5, false, true, 1>;
+// constants only (M <= 128 runs transposed)
 using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
-using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;  // constants only (FP8 M <= 128 runs swapped)
+using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
 using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
-// M <= 128 with few 224-wide tiles: 64-wide tiles put ~3.5x more SMs on the (B-bandwidth-bound)
-// problem, and their 24 KB stages allow a deeper ring.
-using CfgBF16N = GemmCfg<Kind::BF16, 64, 8, false, false>;
-using CfgFP4N = GemmCfg<Kind::FP4, 64, 8, false, false>;
-// FP8 with M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair,
-// A's rows across), written transposed.  Per SM and K step: 128 rows of B and 64 of A (24 KB)
-// for 128 x 128 products, against 24 KB for 128 x 64 in the narrow tiles: half the bytes per
+// M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair, A's rows
+// across), written transposed.  Per SM and K step: 128 rows of B and 64 of A for 128 x 128
+// products, against the same bytes for 128 x 64 in single-CTA narrow tiles: half the bytes per
 // product, in a kernel whose loads are latency-bound.
+using CfgBF16S = GemmCfg<Kind::BF16, 128, 8, false, true, 2, false, true>;
 using CfgFP8S = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true>;
+using CfgFP4S = GemmCfg<Kind::FP4, 128, 7, false, true, 2, false, true>;
 
 // Tile shape by problem shape.  M > 128: CTA pairs, 256 or 224 columns wide, whichever
 // finishes first by a model of the waves (tile time proportional to its MMA work, 224-wide
 // tiles 8% less efficient, a split tail paying for its longest slice plus about four K steps
-// of reduction).  M <= 128: FP8 runs transposed on 256 x 128 pair tiles (swap_small_m); the
-// other kinds use single CTAs, 64 wide when 224-wide tiles would leave most SMs idle.
-enum class Shape { Pair256, Pair224, Wide, Narrow, Swap };
-Shape pick_shape(int M, int N, int num_kb, int period, int sms, bool swap_small_m = false) {
-    if (M <= 128 && swap_small_m) return Shape::Swap;
-    if (M > 128) {
-        const int workers = sms / 2;
-        const auto cost = [&](int bn, double eff) {
-            const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
-            const TailPlan p = plan_tail(tiles, num_kb, period, workers, true);
-            double steps;
-            if (p.splits > 1) {
-                const int groups = (num_kb + period - 1) / period;
-                steps = (double)(p.full_tiles / workers) * num_kb + (double)((groups + p.splits - 1) / p.splits) * period + 4.0;
-            } else {
-                steps = (double)((tiles + workers - 1) / workers) * num_kb;
-            }
-            return steps * 256.0 * bn / eff;
-        };
-        return cost(256, 1.0) <= cost(224, 0.92) ? Shape::Pair256 : Shape::Pair224;
-    }
-    return (N + 223) / 224 * 2 <= sms ? Shape::Narrow : Shape::Wide;
+// of reduction).  M <= 128: the product runs transposed on 256 x 128 pair tiles.
+enum class Shape { Pair256, Pair224, Swap };
+Shape pick_shape(int M, int N, int num_kb, int period, int sms) {
+    if (M <= 128) return Shape::Swap;
+    const int workers = sms / 2;
+    const auto cost = [&](int bn, double eff) {
+        const int tiles = ((M + 255) / 256) * ((N + bn - 1) / bn);
+        const TailPlan p = plan_tail(tiles, num_kb, period, workers, true);
+        double steps;
+        if (p.splits > 1) {
+            const int groups = (num_kb + period - 1) / period;
+            steps = (double)(p.full_tiles / workers) * num_kb + (double)((groups + p.splits - 1) / p.splits) * period + 4.0;
+        } else {
+            steps = (double)((tiles + workers - 1) / workers) * num_kb;
+        }
+        return steps * 256.0 * bn / eff;
+    };
+    return cost(256, 1.0) <= cost(224, 0.92) ? Shape::Pair256 : Shape::Pair224;
 }
 
 // Problem description shared by the GEMM entry points.
@@ -522,7 +517,7 @@ int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
     a.M = M, a.N = N, a.K = K, a.sfb_gran = sfb_gran_n;
     int sms = 0;
     if (device_facts_noalloc(&sms) != BSP_OK) sms = 148;
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, sms, true)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, sms)) {
         case Shape::Pair256: return ScaleChunks<CfgFP8P256>(o, a).bytes();
         case Shape::Pair224: return ScaleChunks<CfgFP8P224>(o, a).bytes();
         default: {  // Swap: M <= 128
@@ -548,7 +543,7 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
     a.M = M, a.N = N, a.K = K;
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx.sms, true)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx.sms)) {
         case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, ctx, stream, scratch, scratch_bytes);
         case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, ctx, stream, scratch, scratch_bytes);
         default: {  // Swap: M <= 128
@@ -585,8 +580,11 @@ int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K, int
     switch (pick_shape(M, N, (K + 63) / 64, CfgBF16::SF_PERIOD, ctx->sms)) {
         case Shape::Pair256: return launch_gemm<CfgBF16P256>(o, a, *ctx, st);
         case Shape::Pair224: return launch_gemm<CfgBF16P224>(o, a, *ctx, st);
-        case Shape::Wide: return launch_gemm<CfgBF16>(o, a, *ctx, st);
-        default: return launch_gemm<CfgBF16N>(o, a, *ctx, st);
+        default: {  // Swap: M <= 128
+            Operands os = o;
+            swap_operands(os, a);
+            return launch_gemm<CfgBF16S>(os, a, *ctx, st);
+        }
     }
 }
 
@@ -612,7 +610,7 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = ldd;
     a.sfb_gran = sfb_gran_n;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx->sms, true)) {
+    switch (pick_shape(M, N, kb, CfgFP8::SF_PERIOD, ctx->sms)) {
         case Shape::Pair256: return launch_gemm<CfgFP8P256>(o, a, *ctx, st);
         case Shape::Pair224: return launch_gemm<CfgFP8P224>(o, a, *ctx, st);
         default: {  // Swap: M <= 128
@@ -645,8 +643,11 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
     switch (pick_shape(M, N, K / 256 + (K % 256 ? 1 : 0), CfgFP4::SF_PERIOD, ctx->sms)) {
         case Shape::Pair256: return launch_gemm<CfgFP4P256>(o, a, *ctx, st);
         case Shape::Pair224: return launch_gemm<CfgFP4P224>(o, a, *ctx, st);
-        case Shape::Wide: return launch_gemm<CfgFP4>(o, a, *ctx, st);
-        default: return launch_gemm<CfgFP4N>(o, a, *ctx, st);
+        default: {  // Swap: M <= 128
+            Operands os = o;
+            swap_operands(os, a);
+            return launch_gemm<CfgFP4S>(os, a, *ctx, st);
+        }
     }
 }
 
@@ -768,11 +769,14 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
             switch (pick_shape(M, N, (K + 63) / 64, CfgBF16::SF_PERIOD, ctx->sms)) {
                 case Shape::Pair256: return describe_plan<CfgBF16P256>(M, N, K, *ctx, plan);
                 case Shape::Pair224: return describe_plan<CfgBF16P224>(M, N, K, *ctx, plan);
-                case Shape::Wide: return describe_plan<CfgBF16>(M, N, K, *ctx, plan);
-                default: return describe_plan<CfgBF16N>(M, N, K, *ctx, plan);
+                default: {  // Swap: M <= 128
+                    BSP_TRY(describe_plan<CfgBF16S>(N, M, K, *ctx, plan));
+                    plan[6] = 1;
+                    return BSP_OK;
+                }
             }
         case 1:
-            switch (pick_shape(M, N, (K + 127) / 128, CfgFP8::SF_PERIOD, ctx->sms, true)) {
+            switch (pick_shape(M, N, (K + 127) / 128, CfgFP8::SF_PERIOD, ctx->sms)) {
                 case Shape::Pair256: return describe_plan<CfgFP8P256>(M, N, K, *ctx, plan);
                 case Shape::Pair224: return describe_plan<CfgFP8P224>(M, N, K, *ctx, plan);
                 default: {  // Swap: M <= 128
@@ -785,8 +789,11 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
             switch (pick_shape(M, N, (K + 255) / 256, CfgFP4::SF_PERIOD, ctx->sms)) {
                 case Shape::Pair256: return describe_plan<CfgFP4P256>(M, N, K, *ctx, plan);
                 case Shape::Pair224: return describe_plan<CfgFP4P224>(M, N, K, *ctx, plan);
-                case Shape::Wide: return describe_plan<CfgFP4>(M, N, K, *ctx, plan);
-                default: return describe_plan<CfgFP4N>(M, N, K, *ctx, plan);
+                default: {  // Swap: M <= 128
+                    BSP_TRY(describe_plan<CfgFP4S>(N, M, K, *ctx, plan));
+                    plan[6] = 1;
+                    return BSP_OK;
+                }
             }
         default: return describe_plan<CfgGrouped>(M, N, K, *ctx, plan);
     }

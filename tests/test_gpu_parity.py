@@ -200,6 +200,15 @@ def test_fp8_small_m_runs_transposed(ops, orc, m, n, k, gran):
     _fp8_case(ops, orc, m, n, k, seed=m * 13 + n, gran=gran)
 
 
+@pytest.mark.parametrize("kind,m,n,k", [("bf16", 128, 3000, 2048), ("bf16", 5, 448, 640), ("fp4", 128, 2000, 4096),
+                                        ("fp4", 40, 704, 1024)])
+def test_bf16_fp4_small_m_run_transposed(ops, orc, kind, m, n, k):
+    plan = ops.gemm_plan(kind, m, n, k)
+    assert plan["transposed"] == 1 and plan["tile_n"] == 128, plan
+    got, ref = _run_kind(ops, kind, m, n, k, seed=m + n)
+    check_gemm(got, ref(orc), f"{kind} small M {m}x{n}x{k} {plan}")
+
+
 # ------------------------------------------------------------------ split last wave
 
 def _run_kind(ops, kind, m, n, k, seed, gran=128, rows=None, cols=None):
@@ -449,9 +458,10 @@ def test_wait_timeout_is_reported_and_context_survives(ops, orc):
 # ------------------------------------------------------------------ tile shapes
 
 @pytest.mark.parametrize("kind", ["fp8", "bf16", "fp4"])
-def test_wide_single_cta_tiles(ops, orc, kind):
-    # M <= 128 with more than 74 tiles of 224 columns: single-CTA 224-wide tiles
+def test_small_m_many_columns(ops, orc, kind):
+    # M <= 128 with N = 16640: 65 transposed pair tiles along N, plus split slices
     m, n, k = 96, 16640, 256
+    assert ops.gemm_plan(kind, m, n, k)["transposed"] == 1
     if kind == "fp8":
         p = inputs.dense_fp8_problem(m, n, k, seed=77)
         D = ops.gemm_fp8_nt(to_dev(p["A"]), to_dev(p["sfa"]), to_dev(p["B"]), to_dev(p["sfb"]))
