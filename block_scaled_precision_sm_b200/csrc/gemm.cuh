@@ -13,9 +13,17 @@
 //   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers and
 //               issues tcgen05.cp of each scale chunk into a rotating TMEM slot and the
 //               tcgen05.mma instructions, committing each stage to its "empty" barrier.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (double-buffered in TMEM so the
-//               next tile's MMAs overlap), round to bf16, stage 32 x 32 blocks in a swizzled
-//               shared-memory buffer (two per warp) and TMA-store them to D.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, round to bf16, stage 32 x 32
+//               blocks in a swizzled shared-memory buffer (two per warp) and TMA-store them to
+//               D.  With two accumulators in TMEM the next tile's MMAs overlap the epilogue;
+//               with one (256-column tiles, whose two accumulators would leave no TMEM for
+//               the scales) the epilogue first drains the whole accumulator into registers.
+//
+// Work items: the persistent workers walk the tiles in raster order; when the last wave would
+// leave most workers idle its tiles are cut along K into slices whose fp32 partial sums are
+// added in slot order (deterministic) by the slices themselves.  The masked grouped layout
+// builds its tile list on the device from the per-expert counts.  TRANS_D configurations
+// compute D^T = B A^T for small M and write the result transposed.
 //
 // PAIR = true: a cluster of two CTAs computes a 256 x BN tile with cta_group::2 MMAs.  CTA r
 // loads A rows [128r, 128r+128) and B rows [r*BN/2, (r+1)*BN/2) of the tile into its own
