@@ -15,10 +15,30 @@ bytes [MN, KB] are converted on the GPU by ``transform_sf_ue8m0``.
 from __future__ import annotations
 
 import ctypes
+import functools
 
 import torch
 
 from . import _lib
+
+
+def _on_tensor_device(fn):
+    """Run `fn` with its tensors' CUDA device current (the library launches on the current
+    device and the current stream); tensors on the CPU or on several devices are refused."""
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        devs = {a.device for a in list(args) + list(kwargs.values()) if isinstance(a, torch.Tensor)}
+        if any(d.type != "cuda" for d in devs):
+            raise ValueError(f"{fn.__name__}: tensors must live on a CUDA device")
+        if len(devs) > 1:
+            raise ValueError(f"{fn.__name__}: tensors on several devices: {sorted(map(str, devs))}")
+        if not devs:
+            return fn(*args, **kwargs)
+        with torch.cuda.device(devs.pop()):
+            return fn(*args, **kwargs)
+
+    return wrapper
 
 
 def _stream(stream=None) -> ctypes.c_void_p:
@@ -51,6 +71,7 @@ def sf_ld(mn: int) -> int:
     return (mn + 7) // 8 * 8
 
 
+@_on_tensor_device
 def transform_sf_ue8m0(sf: torch.Tensor, ld_out: int | None = None, stream=None,
                        out: torch.Tensor | None = None) -> torch.Tensor:
     """fp32 power-of-two scales or uint8 UE8M0 bytes [MN, KB] -> int16 words [ceil(KB/2), ld_out]."""
@@ -79,6 +100,7 @@ def is_packed_sf(sf: torch.Tensor, mn: int, kb: int) -> bool:
             and sf.shape[1] >= mn and sf.stride(1) == 1 and (sf.stride(0) * 2) % 16 == 0)
 
 
+@_on_tensor_device
 def packed_sf(sf: torch.Tensor, mn: int, kb: int, stream=None) -> torch.Tensor:
     """Reuse `sf` if it already is packed, else convert it (fp32 / uint8 [MN, KB])."""
     if is_packed_sf(sf, mn, kb):
@@ -96,6 +118,7 @@ def _out(D, m, n, device):
     return D
 
 
+@_on_tensor_device
 def gemm_bf16_nt(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """D = A * B^T for bf16 A [M, K], B [N, K]."""
     if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
@@ -107,6 +130,7 @@ def gemm_bf16_nt(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor | None = None
     return D
 
 
+@_on_tensor_device
 def gemm_fp8_nt(A, sfa, B, sfb, D=None, sfb_gran_n: int = 128, stream=None) -> torch.Tensor:
     """FP8 E4M3 block-scaled D = A * B^T.  A [M, K], B [N, K] (1-byte dtypes)."""
     A8, B8 = _bytes_u8(A), _bytes_u8(B)
@@ -121,6 +145,7 @@ def gemm_fp8_nt(A, sfa, B, sfb, D=None, sfb_gran_n: int = 128, stream=None) -> t
     return D
 
 
+@_on_tensor_device
 def gemm_fp4_nt(A, sfa, B, sfb, D=None, stream=None) -> torch.Tensor:
     """FP4 E2M1 block-scaled D = A * B^T.  A [M, K/2], B [N, K/2] packed bytes (even K low nibble)."""
     A8, B8 = _bytes_u8(A), _bytes_u8(B)
@@ -135,6 +160,7 @@ def gemm_fp4_nt(A, sfa, B, sfb, D=None, stream=None) -> torch.Tensor:
     return D
 
 
+@_on_tensor_device
 def m_grouped_gemm_fp8_nt_contiguous(A, sfa, B, sfb, m_indices, D=None, sfb_gran_n: int = 128,
                                      stream=None) -> torch.Tensor:
     """M-grouped FP8 GEMM: A [M_total, K], B [G, N, K], sfb packed per expert [G, words, ld]."""
@@ -163,6 +189,7 @@ def m_grouped_gemm_fp8_nt_contiguous(A, sfa, B, sfb, m_indices, D=None, sfb_gran
     return D
 
 
+@_on_tensor_device
 def m_grouped_gemm_fp8_nt_masked(A, sfa, B, sfb, masked_m, D=None, sfb_gran_n: int = 128,
                                  stream=None) -> torch.Tensor:
     """Masked grouped FP8 GEMM: A [G, max_m, K], B [G, N, K], masked_m int32 [G] on the device;
@@ -209,6 +236,7 @@ def kernel_launches() -> int:
     return int(_lib.load().bsp_kernel_launches())
 
 
+@_on_tensor_device
 def quantize_fp8(x: torch.Tensor, block_rows: int = 1, q: torch.Tensor | None = None,
                  sf: torch.Tensor | None = None, stream=None):
     """fp32 / bf16 [rows, cols] -> (E4M3 codes uint8 [rows, cols], SF words int16

@@ -131,3 +131,17 @@ def test_noalloc_scratch_limit_without_gpu(lib):
     # 12000 rows fit: the call gets past the size check (and then fails without a GPU)
     assert lib.gemm_fp8_nt_noalloc(good, good, good, good, good, st, 12000, 7168, 16384, 16384, 16384, 7168,
                                    128, 128, 128, None) != -4
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    from block_scaled_precision_sm_b200 import ops
+
+    a = torch.zeros((128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        ops.gemm_bf16_nt(a, a)
+    with pytest.raises(ValueError, match="CUDA device"):
+        ops.quantize_fp8(torch.zeros((4, 128)), 1)
+    with pytest.raises(ValueError, match="CUDA device"):
+        ops.transform_sf_ue8m0(torch.zeros((4, 2), dtype=torch.uint8))
