@@ -10,7 +10,9 @@
  *     one 16-bit integer, stored MN-major ("DeepSeek lanza kernels de DeepGEMM para
  *     Huawei Ascend 950", section "Qué incluye el lanzamiento"; "DeepGEMM-Ascend cobre
  *     quantas operações no Ascend 950?", section "Fatores de escala FP8 e o formato
- *     UE8M0 no Ascend").
+ *     UE8M0 no Ascend");
+ *   - the masked grouped GEMM the pages list as missing, and the FP8 quantiser that
+ *     produces the GEMM's operands with their scales already in the packed layout.
  *
  * Conventions shared by every call
  *   - "NT": A is M x K row-major (K contiguous), B is N x K row-major, D is M x N
@@ -27,6 +29,11 @@
  *     size a multiple of 16 bytes (the tensor-memory-accelerator copy rule).
  *   - M and N may take any positive value (rows and columns past them are neither
  *     read as data nor written); K has the per-call rule stated below.
+ *   - The GEMM calls take their own scratch (the scale layout for the tensor cores, the
+ *     partial sums of a split last wave) stream-ordered from a pool the library keeps per
+ *     device, and free it on the same stream.  Every call can be captured in a CUDA graph;
+ *     under capture the scratch becomes a graph memory node.
+ *   - Results are deterministic: the same inputs give the same bytes on every run.
  *
  * Packed scale-factor layout ("SF words"): for a matrix with MN scale rows and KB scale
  * blocks along K, the SF tensor is int16 [ceil(KB/2)][ld], with
