@@ -87,3 +87,23 @@ def test_same_seed_same_bytes():
     for key in ("A", "sfa", "B", "sfb"):
         assert np.array_equal(a[key], b[key])
     assert ml_dtypes.float8_e4m3fn  # recipe dependency present
+
+
+def test_masked_problem_layout():
+    p = inputs.masked_fp8_problem(5, 256, 96, 384, seed=3)
+    assert p["A"].shape == (5, 256, 384) and p["B"].shape == (5, 96, 384)
+    assert p["sfa"].shape == (5 * 256, 3) and p["sfb"].shape == (5, 1, 3)
+    assert p["masked_m"].dtype == np.int32 and p["masked_m"].shape == (5,)
+    assert (p["masked_m"] >= 0).all() and (p["masked_m"] <= 256).all()
+    q = inputs.masked_fp8_problem(5, 256, 96, 384, seed=3)
+    assert np.array_equal(p["masked_m"], q["masked_m"]) and np.array_equal(p["A"], q["A"])
+    with pytest.raises(ValueError):
+        inputs.masked_fp8_problem(2, 128, 64, 128, seed=1, counts=[0, 129])
+
+
+def test_normal_matrix_is_seeded_and_rounds_to_bf16():
+    x = inputs.normal_matrix(300, 256, seed=9)
+    assert x.dtype == np.float32 and np.array_equal(x, inputs.normal_matrix(300, 256, seed=9))
+    assert not np.array_equal(x, inputs.normal_matrix(300, 256, seed=10))
+    bits = inputs.normal_matrix(300, 256, seed=9, bf16=True)
+    assert bits.dtype == np.uint16 and np.array_equal(bits, inputs.bf16_operand(x))
