@@ -56,6 +56,14 @@ KERNEL_SOURCES = {
 }
 
 
+def workload_config(world: int) -> dict:
+    """The headline workload, as both arms report it."""
+    return {"workload": "fp8_block_scaled_gemm_nt 4096x7168x16384 (sf transform + gemm)", "M": M, "N": N,
+            "K": K, "sfa": "1x128 ue8m0", "sfb": "128x128 ue8m0",
+            "l2": "flushed by a 1 GiB write before every step, outside the events",
+            "parallelism": f"one independent problem per GPU x{world}"}
+
+
 def gemm_flops(m: int, n: int, k: int) -> float:
     return 2.0 * m * n * k
 
@@ -286,10 +294,7 @@ def run_ours(args):
         "vs_baseline_note": "per-GPU value / the pages' 861 TFLOPS FP8xFP8 at this shape on an Ascend 950DT "
                             "(another machine: context, not the target)",
         "dtype": "e4m3 x ue8m0 scales, fp32 accumulate, bf16 out", "data": "synthetic",
-        "config": {"workload": "fp8_block_scaled_gemm_nt 4096x7168x16384 (sf transform + gemm)", "M": M, "N": N,
-                   "K": K, "sfa": "1x128 ue8m0", "sfb": "128x128 ue8m0",
-                   "l2": "flushed by a 1 GiB write before every step, outside the events",
-                   "parallelism": f"one independent problem per GPU x{world}"},
+        "config": workload_config(world),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} bf16 burst x 2 (nominal fp8/bf16 ratio)",
@@ -557,8 +562,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": "synthetic",
-            "config": {"workload": "fp8_block_scaled_gemm_nt 4096x7168x16384", "M": M, "N": N, "K": K,
-                       "sample_per_step": f"{rows_per_step} rows x {N} columns"},
+            "config": workload_config(world),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": oracle.threads(),
                              "kind": "oracle", "sample": f"{rows_per_step} rows x {N} columns per step"},
             "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
