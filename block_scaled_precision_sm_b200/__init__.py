@@ -5,11 +5,11 @@ this package is its thin Python binding.  There is no CPU fallback: a call witho
 built library or without a B200 raises.
 """
 
-__all__ = ["ops", "lib"]
+__all__ = ["ops", "lib", "shard"]
 
 
 def __getattr__(name):
-    if name in ("ops", "lib"):
+    if name in ("ops", "lib", "shard"):
         import importlib
 
         return importlib.import_module(f".{'_lib' if name == 'lib' else name}", __name__)

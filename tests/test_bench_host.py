@@ -45,3 +45,34 @@ def test_committed_summaries_name_their_command_and_digest():
         text = open(os.path.join(root, "profiles", name)).read()
         assert "ncu " in text and "--clock-control none" in text, name
         assert "sources_digest:" in text, name
+
+
+def test_spread_reports_median_and_percentiles():
+    import numpy as np
+
+    d = bench.spread(np.array([1.0, 2.0, 3.0, 4.0, 100.0]))
+    assert d["median_ms"] == 3.0 and d["samples"] == 5
+    assert d["p10_ms"] < d["median_ms"] < d["p90_ms"] and d["mean_ms"] == 22.0
+
+
+def test_peak_fractions_against_spec_and_clock():
+    # 148 SMs x 16384 FP8 flops per clock at 1965 MHz = 4765 TFLOP/s
+    f = bench.peak_fractions(2382.5, "fp8", 148, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0})
+    assert abs(f["clock_peak_tflops_at_sampled_clock"] - 4764.9) < 0.2
+    assert abs(f["frac_of_clock_peak_at_sampled_clock"] - 0.5) < 1e-3
+    assert f["frac_of_spec"] == round(2382.5 / 4500.0, 4)
+    assert "frac_of_clock_peak_at_sampled_clock" not in bench.peak_fractions(1.0, "bf16", 148, {"sm_mhz": None})
+
+
+def test_clock_window_selects_the_timed_samples(monkeypatch):
+    s = bench.ClockSampler(0)
+    s.max_mhz = 1965.0
+    sw_power_cap = 0x4
+    s.samples = [(0.0, 1000.0, 100.0, 0), (1.0, 1965.0, 500.0, 0), (1.001, 1950.0, 600.0, sw_power_cap),
+                 (1.002, 1965.0, 550.0, 0), (2.0, 900.0, 90.0, 0)]
+    w = s.window(0.9, 1.1)
+    assert w["samples"] == 3 and w["sm_mhz"] == 1965.0 and w["sm_mhz_min"] == 1950.0
+    assert w["reasons"] == ["sw_power_cap"]
+    # a window shorter than the sampling period takes the samples on either side
+    assert s.window(1.5, 1.6)["samples"] == 2
+    assert bench.ClockSampler(0).window()["samples"] == 0
