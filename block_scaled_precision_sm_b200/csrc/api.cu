@@ -5,6 +5,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -35,6 +36,18 @@ struct DeviceCtx {
 std::mutex g_mu;
 DeviceCtx g_dev[kMaxDevices];
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+// K steps the GEMMs' L2 prefetch of operand tiles runs ahead of their loads; the environment
+// variable BSP_L2_PREFETCH_KSTEPS, read once, overrides it (0 turns the prefetch off).
+constexpr int kDefaultPrefetchKSteps = 8;
+int prefetch_ksteps() {
+    static const int v = [] {
+        const char* e = std::getenv("BSP_L2_PREFETCH_KSTEPS");
+        const int x = e ? std::atoi(e) : kDefaultPrefetchKSteps;
+        return x < 0 ? 0 : (x > 64 ? 64 : x);
+    }();
+    return v;
+}
 std::atomic<uint64_t> g_launches{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -139,8 +152,8 @@ int max_workers_of(const DeviceCtx& ctx, int* out) {
 
 // Tail plan: how many whole tiles, and into how many K slices the rest is cut.  The tiles
 // left over after the last full wave of workers are split when at least two slices of
-// eight or more K steps fit per tile, up to 16 slices (a power of two), so that the last
-// wave keeps most workers busy instead of a few.
+// eight or more K steps fit per tile, up to 16 slices and no more than the idle workers
+// take in one wave, so that the last wave keeps most workers busy instead of a few.
 struct TailPlan {
     int tiles, full_tiles, splits, tail_tiles, num_work;
 };
@@ -154,7 +167,6 @@ TailPlan plan_tail(int tiles, int num_kb, int period, int workers, bool allow) {
     s = s < 16 ? s : 16;
     s = s < groups ? s : groups;
     while (s >= 2 && num_kb / s < 8) --s;
-    while (s & (s - 1)) --s;  // a power of two: every slice then sums 32/S rows of each warp
     if (s < 2) return p;
     p.full_tiles = tiles - rem;
     p.splits = s;
@@ -167,9 +179,15 @@ template <class C>
 int64_t tail_ws_bytes(const TailPlan& p) {
     return p.splits > 1 ? (int64_t)p.tail_tiles * p.splits * C::TILE_M * C::BN * 4 : 0;
 }
+// Split-tail counters ([split tiles][CTAs][4 epilogue warps] int) followed by the share
+// claims ([split tiles][CTAs][4][splits] int), zeroed before the GEMM runs.
+template <class C>
+int64_t tail_counters(const TailPlan& p) {
+    return (int64_t)p.tail_tiles * C::CTAS * 4;
+}
 template <class C>
 int64_t tail_count_bytes(const TailPlan& p) {
-    return p.splits > 1 ? round_up_i((int64_t)p.tail_tiles * C::CTAS * 4 * 4, 256) : 0;
+    return p.splits > 1 ? round_up_i(tail_counters<C>(p) * (1 + p.splits) * 4, 256) : 0;
 }
 
 // Launch config C with the split-tail plan `p` (ws: its workspace, count: its zeroed counters).
@@ -201,9 +219,11 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     a.num_work = p.num_work;
     a.ws = ws;
     a.tail_count = count;
+    a.tail_claim = count ? count + tail_counters<C>(p) : nullptr;
     a.group_m = 16;
     a.status = ctx.status;
     a.timeout_ns = g_timeout_ns.load();
+    a.prefetch = prefetch_ksteps();
     const int workers = a.num_work < max_workers ? a.num_work : max_workers;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -241,6 +261,9 @@ using CfgBF16 = GemmCfg<Kind::BF16, 224, 4, false, false>;
 using CfgFP8 = GemmCfg<Kind::FP8, 224, 4, false, false>;
 using CfgFP4 = GemmCfg<Kind::FP4, 224, 4, false, false>;
 using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
+// contiguous grouped layout on CTA pairs (pairs of 128-row blocks of one expert), used while the
+// block count fits the kernel's on-device tile list; CfgGrouped (single CTAs) otherwise
+using CfgGroupedPair = GemmCfg<Kind::FP8, 224, 6, true, true>;
 using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 // M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair, A's rows
 // across), written transposed.  Per SM and K step: 128 rows of B and 64 of A for 128 x 128
@@ -362,15 +385,16 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, pools[dev], stream) == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
 }
 
-// Chunk tensor map: 8-byte elements, one chunk per (row tile, group [, expert]).
-int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int q, int experts_or_neg) {
+// Chunk tensor map: 8-byte elements, one chunk per (row tile, group [, expert]); a box is the
+// chunks of `batch` consecutive groups of one row tile (groups past the last read as zeros).
+int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int q, int experts_or_neg, int batch) {
     // experts_or_neg < 0: a rank-4 map over -experts_or_neg experts (the grouped kernel's 4-D loads)
     const int experts = experts_or_neg < 0 ? -experts_or_neg : experts_or_neg;
     const cuuint64_t dims[4] = {(cuuint64_t)(chunk_bytes / 8), (cuuint64_t)tiles, (cuuint64_t)q,
                                 (cuuint64_t)experts};
     const cuuint64_t strides[3] = {(cuuint64_t)chunk_bytes, (cuuint64_t)chunk_bytes * tiles,
                                    (cuuint64_t)chunk_bytes * tiles * q};
-    const cuuint32_t box[4] = {(cuuint32_t)(chunk_bytes / 8), 1, 1, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)(chunk_bytes / 8), 1, (cuuint32_t)batch, 1};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, experts_or_neg < 0 ? 4 : 3, base, dims, strides, box,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
@@ -385,6 +409,11 @@ int plan_gemm(GemmArgs& a, const DeviceCtx& ctx, TailPlan* p, int* workers) {
     int max_workers = 0;
     BSP_TRY(max_workers_of<C>(ctx, &max_workers));
     *p = plan_tail(a.m_blocks * a.n_blocks, a.num_kb, C::SF_PERIOD, max_workers, !C::GROUPED);
+    if constexpr (C::PAIR_LIST) {
+        // the pair tiles are found on the device: between M/256 and M/128 of them per column block;
+        // the grid is sized for the most
+        p->tiles = p->full_tiles = p->num_work = (a.M / 128) * a.n_blocks;
+    }
     *workers = max_workers;
     return BSP_OK;
 }
@@ -449,8 +478,9 @@ int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_
         char* wa = base;
         char* wb = wa + ScaleChunks<C>(o, a).a_bytes;
         rc = launch_sf_layout(o.sfa, la, wa, o.sfb, lb, wb, count, tail_bytes ? tail_count_bytes<C>(p) : 0, stream);
-        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1);
-        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1);
+        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1, C::SF_BATCH);
+        if (rc == BSP_OK)
+            rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1, C::SF_BATCH);
     } else {
         tsa = ta, tsb = tb;  // not read
         if (tail_bytes && cudaMemsetAsync(count, 0, (size_t)tail_count_bytes<C>(p), stream) != cudaSuccess)
@@ -503,11 +533,10 @@ void note_launch() { g_launches.fetch_add(1); }
 
 int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
                            cudaStream_t stream) {
-    const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
-    if (grid.y > 65535u) return BSP_ERR_UNSUPPORTED;
-    sf_transform_kernel<1><<<grid, 256, 0, stream>>>(in, mn, kb, ld_in, static_cast<uint16_t*>(out), ld_out, status);
+    if ((kb + kSfTileKB - 1) / kSfTileKB > 65535) return BSP_ERR_UNSUPPORTED;
+    const bool ok = launch_sf_transform(in, 1, mn, kb, ld_in, static_cast<uint16_t*>(out), ld_out, status, stream);
     g_launches.fetch_add(1);
-    return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
+    return ok ? BSP_OK : BSP_ERR_CUDA;
 }
 
 int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n) {
@@ -674,6 +703,8 @@ int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void*
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = N;
     a.m_indices = m_indices, a.G = G;
     a.sfb_gran = sfb_gran_n;
+    if (M_total / 128 <= CfgGroupedPair::MAX_PAIR_TILES)
+        return launch_gemm<CfgGroupedPair>(o, a, *ctx, static_cast<cudaStream_t>(stream));
     return launch_gemm<CfgGrouped>(o, a, *ctx, static_cast<cudaStream_t>(stream));
 }
 
@@ -718,18 +749,13 @@ int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t l
     const char* ob = static_cast<const char*>(sf_out);
     const char* oe = ob + (int64_t)words * ld_out * 2;
     if (ib < oe && ob < ie) return BSP_ERR_ARG;  // overlapping buffers
+    if ((kb + kSfTileKB - 1) / kSfTileKB > 65535) return BSP_ERR_UNSUPPORTED;
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
-    const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
-    if (grid.y > 65535u) return BSP_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint16_t* out = static_cast<uint16_t*>(sf_out);
-    if (in_kind == 0)
-        sf_transform_kernel<0><<<grid, 256, 0, st>>>(sf_in, mn, kb, ld_in, out, ld_out, ctx->status);
-    else
-        sf_transform_kernel<1><<<grid, 256, 0, st>>>(sf_in, mn, kb, ld_in, out, ld_out, ctx->status);
+    const bool ok = launch_sf_transform(sf_in, in_kind, mn, kb, ld_in, static_cast<uint16_t*>(sf_out), ld_out,
+                                        ctx->status, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1);
-    return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
+    return ok ? BSP_OK : BSP_ERR_CUDA;
 }
 
 int bsp_get_device_status(void* stream) {
@@ -795,7 +821,9 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                     return BSP_OK;
                 }
             }
-        default: return describe_plan<CfgGrouped>(M, N, K, *ctx, plan);
+        default:
+            if (M / 128 <= CfgGroupedPair::MAX_PAIR_TILES) return describe_plan<CfgGroupedPair>(M, N, K, *ctx, plan);
+            return describe_plan<CfgGrouped>(M, N, K, *ctx, plan);
     }
 }
 

@@ -7,12 +7,13 @@
 // operandos e pipelining na prática", rebuilt for Blackwell):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) into an S-stage shared-memory
 //               ring ("full"/"empty" mbarriers, transaction-counted); the first stage of every
-//               scale group (SF_PERIOD K steps) also carries one chunk of scale words per
-//               operand, laid out beforehand (sf_layout.cuh) exactly as the scale copy reads
+//               batch of SF_BATCH scale groups (SF_PERIOD K steps each) also carries the
+//               batch's chunks of scale words into a two-slot scale ring (released by its own
+//               barriers), laid out beforehand (sf_layout.cuh) exactly as the scale copy reads
 //               them, so no thread rearranges scales on chip.
-//   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers and
-//               issues tcgen05.cp of each scale chunk into a rotating TMEM slot and the
-//               tcgen05.mma instructions, committing each stage to its "empty" barrier.
+//   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers, issues
+//               one burst of tcgen05.cp per batch (every group's chunks into its own TMEM slot)
+//               and the tcgen05.mma instructions, committing each stage to its "empty" barrier.
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, round to bf16, stage 32 x 32
 //               blocks in a swizzled shared-memory buffer (two per warp) and TMA-store them to
 //               D.  With two accumulators in TMEM the next tile's MMAs overlap the epilogue;
@@ -21,7 +22,8 @@
 //
 // Work items: the persistent workers walk the tiles in raster order; when the last wave would
 // leave most workers idle its tiles are cut along K into slices whose fp32 partial sums are
-// added in slot order (deterministic) by the slices themselves.  The masked grouped layout
+// added in slot order (deterministic) by the slices themselves, without any slice waiting on
+// another that may not be resident.  The masked grouped layout
 // builds its tile list on the device from the per-expert counts.  TRANS_D configurations
 // compute D^T = B A^T for small M and write the result transposed.
 //
@@ -71,18 +73,21 @@ struct GemmArgs {
     unsigned long long timeout_ns;
     // Split tail: the first full_tiles tiles (in raster order) are computed whole, one per
     // work item; each remaining tile is cut into `splits` slices along K.  Slice j stores its
-    // fp32 partial sums in its own workspace slot (ws: [split tiles][splits][TILE_M][BN]),
-    // counts itself in tail_count ([split tiles][CTAs][4 epilogue warps], zero on entry) and
-    // waits for the other slices; then slice j adds up all slots, in slot order, for its
-    // share of the rows and rounds them to bf16 in D.  The fixed order keeps the result
-    // identical from run to run.
+    // fp32 partial sums in its own workspace slot (ws: [split tiles][splits][TILE_M][BN]) and
+    // counts itself in tail_count ([split tiles][CTAs][4 epilogue warps], zero on entry); the
+    // rows of each epilogue warp are cut into `splits` shares, each claimed once through
+    // tail_claim ([split tiles][CTAs][4][splits], zero on entry) and summed over all slots in
+    // slot order before the bf16 rounding.  The fixed order keeps the result identical from
+    // run to run, whichever slice reduces a share.
     int full_tiles;
     int splits;
     int num_work;  // full_tiles + (num_tiles - full_tiles) * splits
     float* ws;
     int* tail_count;
+    int* tail_claim;
     const int32_t* masked_m;  // masked layout: valid rows per expert [G]
     int max_m;                // masked layout: rows per expert slab
+    int prefetch;             // K steps the L2 prefetch of A and B runs ahead of the loads (0: off)
 };
 
 template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false,
@@ -102,6 +107,11 @@ struct GemmCfg {
     static constexpr bool MASKED = MASKED_;
     static constexpr int MAX_MASKED_G = 1024;
     static_assert(!MASKED || (GROUPED && !PAIR_), "masked layout: single-CTA grouped configs only");
+    // contiguous grouped layout on CTA pairs: a pair tile is one or two consecutive 128-row blocks
+    // of one expert (an expert's odd last block alone, its peer CTA's rows then not stored); the
+    // list of pair tiles is built on the device at kernel start from the blocks' expert indices
+    static constexpr bool PAIR_LIST = GROUPED && PAIR_ && !MASKED;
+    static constexpr int MAX_PAIR_TILES = 2048;
     // the kernel computes D^T = B' A'^T with the caller's operands swapped (A' = B, B' = A) and
     // writes each accumulator element (row i, column j) to D[j][i]: small-M problems put the
     // long N dimension on the 256-row pair tiles
@@ -128,32 +138,48 @@ struct GemmCfg {
     static constexpr int SFB_CHUNK = SCALED ? SFB_ATOMS * UT_WORDS * 512 : 0;
     static constexpr int SF_STAGE_BYTES = SFA_CHUNK + SFB_CHUNK;
 
-    // Tensor memory: ACC_BUFS fp32 accumulators of BN columns, then rotating scale slots.
+    // Tensor memory: ACC_BUFS fp32 accumulators of BN columns, then the scale slots.  Scales
+    // reach tensor memory in batches of SF_BATCH groups (one burst of copies per batch, so the
+    // tensor pipe switches between copies and MMAs once per batch instead of once per group),
+    // into two sets of SF_BATCH slots used alternately: batch b is copied while the MMAs of
+    // batch b - 1 may still read the other set.
     static constexpr int TMEM_COLS = 512;
     static constexpr int ACC_COLS = ACC_BUFS * BN;
     static constexpr int SFA_COLS = UT_WORDS * 4;
     static constexpr int SFB_COLS = UT_WORDS * SFB_ATOMS * 4;
     static constexpr int SF_SLOT_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int SF_SLOTS_FIT = SCALED ? (TMEM_COLS - ACC_COLS) / SF_SLOT_COLS : 1;
-    static constexpr int SF_SLOTS = SF_SLOTS_FIT > 4 ? 4 : SF_SLOTS_FIT;
-    static_assert(!SCALED || SF_SLOTS >= 1, "tensor memory too small for the scale slots");
+    static constexpr int SF_BATCH = !SCALED                                         ? 1
+                                    : ACC_COLS + 8 * SF_SLOT_COLS <= TMEM_COLS ? 4
+                                    : ACC_COLS + 4 * SF_SLOT_COLS <= TMEM_COLS ? 2
+                                                                               : 1;
+    static constexpr int SF_SLOTS = 2 * SF_BATCH;
+    static_assert(!SCALED || ACC_COLS + SF_SLOTS * SF_SLOT_COLS <= TMEM_COLS,
+                  "tensor memory too small for the scale slots");
+    static constexpr int SF_BATCH_KSTEPS = SF_BATCH * SF_PERIOD;  // K steps per batch
+    static constexpr int SF_BATCH_BYTES = SF_BATCH * SF_STAGE_BYTES;
 
     // Shared memory map (offsets from a 1024-byte aligned base).
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;  // a scale chunk buffer per stage
+    // scale ring: two batches of chunks (A chunks of the batch's groups, then B chunks), each
+    // loaded with the first A/B stage of its batch and released by its own barrier
+    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
     // epilogue staging: per epilogue warp two 32 x 32 bf16 blocks (64-byte swizzle)
     static constexpr int EPI_BLOCK = 32 * 32 * 2;
-    static constexpr int OFF_EPI = ((OFF_SF + STAGES * SF_STAGE_BYTES + 1023) / 1024) * 1024;
-    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain
-    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail gather
-    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
+    static constexpr int OFF_EPI = ((OFF_SF + (SCALED ? 2 * SF_BATCH_BYTES : 0) + 1023) / 1024) * 1024;
+    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail
+    // gather [4]; scale ring empty [2]
+    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4 + 2;
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // masked layout: valid m-blocks before each expert [G + 1] and the clamped counts [G]
     static constexpr int OFF_MASK = OFF_MISC + 16;
     static constexpr int MASK_BYTES = MASKED ? (2 * MAX_MASKED_G + 1) * 4 : 0;
-    static constexpr int SMEM_BYTES = OFF_MASK + MASK_BYTES + 1024;  // + alignment slack
+    // pair-tile list of the contiguous grouped layout: [MAX_PAIR_TILES] entries, then the count
+    static constexpr int OFF_LIST = OFF_MASK + MASK_BYTES;
+    static constexpr int LIST_BYTES = PAIR_LIST ? (MAX_PAIR_TILES + 1) * 4 : 0;
+    static_assert(!PAIR_LIST || MAX_PAIR_TILES * 4 <= STAGES * A_BYTES, "block expert scratch");
+    static constexpr int SMEM_BYTES = OFF_LIST + LIST_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     // a K slice of a split tile is a worker's last work item, so its epilogue stages the
     // fp32 partial sums (BM x BN) in the then idle A/B stage buffers
@@ -201,6 +227,63 @@ __device__ __forceinline__ void masked_tile(const GemmArgs& a, const int* mprefi
     *m0 = lo * a.max_m + (mbi - mprefix[lo]) * 128;
 }
 
+// Contiguous grouped layout on CTA pairs: the pair tiles, built by one warp of each CTA.  A
+// block of 128 rows belongs to the expert of its first row (e[b] = m_indices[128 b]); a run of
+// blocks of one expert is cut into pairs from its first block on, an odd last block forming a
+// tile of its own.  Entry i of `list` is the tile's first block | (its block count << 24);
+// list[max_tiles] is the count.  `e` is scratch for the blocks' experts (M / 128 ints).
+__device__ __forceinline__ void build_pair_list(const GemmArgs& a, int* e, int* list, int max_tiles, uint32_t lane) {
+    const int nb = a.M / 128;
+    for (int b = (int)lane; b < nb; b += 32) e[b] = __ldg(a.m_indices + (int64_t)b * 128);
+    __syncwarp();
+    const int per = (nb + 31) / 32;
+    const int c0 = min(nb, (int)lane * per), c1 = min(nb, c0 + per);
+    const auto run_start = [&](int b) { return b == 0 || e[b] != e[b - 1]; };
+    // the run start in effect where this lane's blocks begin: the last one of earlier lanes
+    int last = -1;
+    for (int b = c0; b < c1; ++b)
+        if (run_start(b)) last = b;
+    int incl = last;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if ((int)lane >= o) incl = max(incl, v);
+    }
+    int carry = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) carry = 0;
+    // a block starts a tile when it lies an even number of blocks after its run's start
+    int rs = carry, count = 0;
+    for (int b = c0; b < c1; ++b) {
+        if (run_start(b)) rs = b;
+        count += ((b - rs) & 1) == 0;
+    }
+    int pos = count;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, pos, o);
+        if ((int)lane >= o) pos += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, pos, 31);
+    pos -= count;
+    rs = carry;
+    for (int b = c0; b < c1; ++b) {
+        if (run_start(b)) rs = b;
+        if (((b - rs) & 1) == 0) {
+            const int len = (b + 1 < nb && e[b + 1] == e[b]) ? 2 : 1;
+            if (pos < max_tiles) list[pos] = b | (len << 24);
+            ++pos;
+        }
+    }
+    if (lane == 0) list[max_tiles] = min(total, max_tiles);
+}
+
+__device__ __forceinline__ void pair_tile(const GemmArgs& a, const int* list, int w, int* b0, int* len, int* n_blk) {
+    const int i = w / a.n_blocks;
+    *n_blk = w - i * a.n_blocks;
+    *b0 = list[i] & 0xFFFFFF;
+    *len = list[i] >> 24;
+}
+
 __device__ __forceinline__ Tile tile_of(const GemmArgs& a, int t) {
     const int per_group = a.group_m * a.n_blocks;
     const int grp = t / per_group;
@@ -240,6 +323,12 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, con
 // before its own copies and MMAs (which finish in microseconds) have landed.
 constexpr unsigned long long kDrainTimeoutNs = 1000000000ull;
 
+// How long a slice of a split tile looks for the other slices of its tile to publish before it
+// leaves the reduction of its share to the slice that publishes last.  The slices of a tile
+// normally finish within a few microseconds of one another; one that is not resident (its SM
+// held by another kernel) arrives later, and then reduces every open share itself.
+constexpr unsigned long long kTailPollNs = 40000ull;
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const GemmArgs& a) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -274,6 +363,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* tmem_empty = tmem_full + 2;
     uint64_t* drain = tmem_empty + 2;
     uint64_t* gather = drain + 1;  // [4]: one per epilogue warp
+    uint64_t* sf_empty = gather + 4;  // [2]: scale ring slots
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -296,6 +386,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mbar_init(drain, 1);
         for (int w = 0; w < 4; ++w) mbar_init(&gather[w], 1);
+        for (int b = 0; b < 2; ++b) mbar_init(&sf_empty[b], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -350,6 +441,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (lane == 31) mprefix[G] = incl;
         }
     }
+    int* plist = reinterpret_cast<int*>(smem + C::OFF_LIST);
+    if constexpr (C::PAIR_LIST) {
+        // the A stage buffers are idle until the setup barrier below: scratch for the blocks' experts
+        if (warp == 2) build_pair_list(args, reinterpret_cast<int*>(smem + C::OFF_A), plist, C::MAX_PAIR_TILES, lane);
+    }
     tc_fence_before();
     if constexpr (C::PAIR)
         cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
@@ -357,32 +453,82 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
-    const int num_work = C::MASKED ? mprefix[args.G] * args.n_blocks : args.num_work;
+    const int num_work = C::MASKED      ? mprefix[args.G] * args.n_blocks
+                         : C::PAIR_LIST ? plist[C::MAX_PAIR_TILES] * args.n_blocks
+                                        : args.num_work;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t it = 0;
+            uint32_t it = 0, bc = 0;  // K steps and scale batches issued
             bool ok = true;
             bool prior_done = false;  // the scale chunks come from the kernel launched before
-            for (int w = worker; w < num_work && ok; w += workers) {
-                Work wk{0, 0, args.num_kb, -1, 0};
-                int m0, n_blk, g = 0;
+            // this CTA's rows of work item w: its K range, first A row, tile column and expert
+            struct Item {
+                Work wk;
+                int m0, n_blk, g;
+            };
+            const auto item_of = [&](int w, bool check) {
+                Item t{Work{0, 0, args.num_kb, -1, 0}, 0, 0, 0};
                 if constexpr (C::MASKED) {
-                    masked_tile(args, mprefix, w, &m0, &n_blk, &g);
+                    masked_tile(args, mprefix, w, &t.m0, &t.n_blk, &t.g);
+                } else if constexpr (C::PAIR_LIST) {
+                    int b0, len;
+                    pair_tile(args, plist, w, &b0, &len, &t.n_blk);
+                    t.m0 = (b0 + (int)rank) * C::BM;
+                    t.g = __ldg(args.m_indices + (int64_t)b0 * C::BM);  // both CTAs multiply by this expert's B
+                    if (t.g < 0 || t.g >= args.G) {
+                        if (check) latch_status(args.status, kStatusDeviceCheck);
+                        t.g = 0;
+                    }
                 } else {
-                    wk = work_of(args, w, C::SF_PERIOD);
-                    const Tile tl = tile_of(args, wk.tile);
-                    m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
-                    n_blk = tl.n_blk;
+                    t.wk = work_of(args, w, C::SF_PERIOD);
+                    const Tile tl = tile_of(args, t.wk.tile);
+                    t.m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
+                    t.n_blk = tl.n_blk;
                     if constexpr (C::GROUPED) {
-                        g = __ldg(args.m_indices + m0);
-                        if (g < 0 || g >= args.G) {
-                            latch_status(args.status, kStatusDeviceCheck);
-                            g = 0;
+                        t.g = __ldg(args.m_indices + t.m0);
+                        if (t.g < 0 || t.g >= args.G) {
+                            if (check) latch_status(args.status, kStatusDeviceCheck);
+                            t.g = 0;
                         }
                     }
                 }
+                return t;
+            };
+            // L2 prefetch: a cursor runs args.prefetch K steps ahead of the loads, across work
+            // items, and brings the A and B boxes of its K step into L2 (no shared memory), so
+            // that a load finds its tile in L2 instead of waiting for DRAM
+            int pw = worker, pkb = 0;
+            Item pt{};
+            bool pvalid = args.prefetch > 0 && worker < num_work;
+            if (pvalid) {
+                pt = item_of(pw, false);
+                pkb = pt.wk.kb0;
+            }
+            const auto prefetch_next = [&] {
+                if (!pvalid) return;
+                const int px = pkb * (C::kind == Kind::BF16 ? 64 : 128);
+                const int pnb0 = pt.n_blk * C::BN + (int)rank * C::BN_CTA;
+                tma_prefetch_2d(&tm_a, px, pt.m0);
+                if constexpr (C::GROUPED)
+                    tma_prefetch_3d(&tm_b, px, pnb0, pt.g);
+                else
+                    tma_prefetch_2d(&tm_b, px, pnb0);
+                if (++pkb >= pt.wk.kb1) {
+                    pw += workers;
+                    pvalid = pw < num_work;
+                    if (pvalid) {
+                        pt = item_of(pw, false);
+                        pkb = pt.wk.kb0;
+                    }
+                }
+            };
+            for (int i = 0; i < args.prefetch; ++i) prefetch_next();
+            for (int w = worker; w < num_work && ok; w += workers) {
+                const Item cur = item_of(w, true);
+                const Work wk = cur.wk;
+                const int m0 = cur.m0, n_blk = cur.n_blk, g = cur.g;
                 const int n0 = n_blk * C::BN;
                 const int nb0 = n0 + (int)rank * C::BN_CTA;
                 for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
@@ -392,13 +538,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    const bool sf_here = C::SCALED && kb % C::SF_PERIOD == 0;
+                    // the first K step of every batch of scale groups also brings the batch's chunks
+                    const bool sf_here = C::SCALED && (kb - wk.kb0) % C::SF_BATCH_KSTEPS == 0;
+                    if (sf_here && !bounded_wait(&sf_empty[bc & 1u], ((bc >> 1) & 1u) ^ 1u, args, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     if (leader)
                         mbar_arrive_expect_tx(&full[s], C::CTAS * (C::A_BYTES + C::B_BYTES +
-                                                                   (sf_here ? C::SF_STAGE_BYTES : 0)));
+                                                                   (sf_here ? C::SF_BATCH_BYTES : 0)));
                     uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
                     uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-                    uint8_t* sf = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
+                    uint8_t* sf = smem + C::OFF_SF + (bc & 1u) * C::SF_BATCH_BYTES;
+                    if (sf_here) ++bc;
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
                     const int q = kb / C::SF_PERIOD;
@@ -409,11 +561,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if constexpr (C::PAIR) {
                         const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), 0);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
-                        tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
+                        if constexpr (C::GROUPED)
+                            tma_load_3d_pair(sb, &tm_b, lead_full, kx, nb0, g);
+                        else
+                            tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
                         if (sf_here) {
-                            // scale chunks: this CTA's A rows, all BN B rows of the tile
+                            // scale chunks of the batch's groups: this CTA's A rows, all BN B rows of the tile
                             tma_load_3d_pair(sf, &tm_sfa, lead_full, 0, m0 / C::BM, q);
-                            tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q);
+                            if constexpr (C::GROUPED)
+                                tma_load_4d_pair(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q, g);
+                            else
+                                tma_load_3d_pair(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q);
                         }
                     } else {
                         tma_load_2d(sa, &tm_a, &full[s], kx, m0);
@@ -424,11 +582,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (sf_here) {
                             tma_load_3d(sf, &tm_sfa, &full[s], 0, m0 / C::BM, q);
                             if constexpr (C::GROUPED)
-                                tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q, g);
+                                tma_load_4d(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q, g);
                             else
-                                tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q);
+                                tma_load_3d(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q);
                         }
                     }
+                    prefetch_next();
                 }
             }
             // Wind down: wait (bounded) until the copies issued for the last stages landed.
@@ -442,10 +601,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == 1 && leader) {
         // ------------------------------------------------------------ MMA issue (one lane)
         if (lane == 0) {
-            uint32_t it = 0, lt = 0, git = 0;
+            uint32_t it = 0, lt = 0, bc = 0;  // K steps, work items and scale batches issued
             bool ok = true;
             for (int w = worker; w < num_work && ok; w += workers, ++lt) {
-                const Work wk = C::MASKED ? Work{0, 0, args.num_kb, -1, 0} : work_of(args, w, C::SF_PERIOD);
+                const Work wk =
+                    (C::MASKED || C::PAIR_LIST) ? Work{0, 0, args.num_kb, -1, 0} : work_of(args, w, C::SF_PERIOD);
                 const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
                 const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
                 if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
@@ -454,7 +614,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * C::BN;
-                uint32_t slot = 0;
+                uint32_t slot = 0, slot_base = 0;
                 for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
@@ -464,33 +624,47 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     tc_fence_after();
                     if constexpr (C::SCALED) {
-                        if (kb % C::SF_PERIOD == 0) {
-                            // copy this group's scale chunks (carried by this stage) into TMEM slot
-                            // git % SF_SLOTS; copies and MMAs run in issue order on the tensor pipe
-                            slot = git % C::SF_SLOTS;
-                            ++git;
-                            const uint32_t sfa_col = C::ACC_COLS + slot * C::SF_SLOT_COLS;
-                            const uint32_t sfb_col = sfa_col + C::SFA_COLS;
-                            const uint8_t* ua = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
-                            const uint8_t* ub = ua + C::SFA_CHUNK;
+                        const int rel = kb - wk.kb0;
+                        if (rel % C::SF_BATCH_KSTEPS == 0) {
+                            // copy the chunks of this batch's groups (carried in with this stage) into
+                            // the slot set bc % 2, one slot per group; copies and MMAs run in issue
+                            // order on the tensor pipe, so the MMAs that read the set two batches ago
+                            // were done before these copies overwrite it
+                            slot_base = (bc & 1u) * C::SF_BATCH;
+                            const uint8_t* sf = smem + C::OFF_SF + (bc & 1u) * C::SF_BATCH_BYTES;
 #pragma unroll
-                            for (int u = 0; u < C::UT_WORDS; ++u) {
-                                if constexpr (C::PAIR)
-                                    tc_cp_32x128b_warpx4_pair(tmem_base + sfa_col + 4 * u,
-                                                              smem_desc_rows16(ua + u * 512));
-                                else
-                                    tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(ua + u * 512));
+                            for (int i = 0; i < C::SF_BATCH; ++i) {
+                                if (kb + i * C::SF_PERIOD >= wk.kb1) break;
+                                const uint32_t sfa_col = C::ACC_COLS + (slot_base + i) * C::SF_SLOT_COLS;
+                                const uint32_t sfb_col = sfa_col + C::SFA_COLS;
+                                const uint8_t* ua = sf + i * C::SFA_CHUNK;
+                                const uint8_t* ub = sf + C::SF_BATCH * C::SFA_CHUNK + i * C::SFB_CHUNK;
 #pragma unroll
-                                for (int at = 0; at < C::SFB_ATOMS; ++at) {
-                                    const uint32_t col = tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at);
-                                    const uint64_t d = smem_desc_rows16(ub + (at * C::UT_WORDS + u) * 512);
+                                for (int u = 0; u < C::UT_WORDS; ++u) {
                                     if constexpr (C::PAIR)
-                                        tc_cp_32x128b_warpx4_pair(col, d);
+                                        tc_cp_32x128b_warpx4_pair(tmem_base + sfa_col + 4 * u,
+                                                                  smem_desc_rows16(ua + u * 512));
                                     else
-                                        tc_cp_32x128b_warpx4(col, d);
+                                        tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(ua + u * 512));
+#pragma unroll
+                                    for (int at = 0; at < C::SFB_ATOMS; ++at) {
+                                        const uint32_t col = tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at);
+                                        const uint64_t d = smem_desc_rows16(ub + (at * C::UT_WORDS + u) * 512);
+                                        if constexpr (C::PAIR)
+                                            tc_cp_32x128b_warpx4_pair(col, d);
+                                        else
+                                            tc_cp_32x128b_warpx4(col, d);
+                                    }
                                 }
                             }
+                            // the ring slot is free once these copies (and the MMAs before them) are done
+                            if constexpr (C::PAIR)
+                                tc_commit_pair_mc(&sf_empty[bc & 1u], kPairMask);
+                            else
+                                tc_commit(&sf_empty[bc & 1u]);
+                            ++bc;
                         }
+                        slot = slot_base + (uint32_t)((rel % C::SF_BATCH_KSTEPS) / C::SF_PERIOD);
                     }
                     const uint64_t adesc = smem_desc_k_sw128(smem + C::OFF_A + s * C::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + s * C::B_BYTES);
@@ -554,8 +728,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int w = worker; w < num_work; w += workers, ++lt) {
             Work wk{0, 0, args.num_kb, -1, 0};
             int m0, n_blk, g = 0;
+            bool mine = true;  // this CTA's rows belong to the tile (false: the peer half of a one-block pair tile)
             if constexpr (C::MASKED) {
                 masked_tile(args, mprefix, w, &m0, &n_blk, &g);
+            } else if constexpr (C::PAIR_LIST) {
+                int b0, len;
+                pair_tile(args, plist, w, &b0, &len, &n_blk);
+                m0 = (b0 + (int)rank) * C::BM;
+                mine = (int)rank < len;
             } else {
                 wk = work_of(args, w, C::SF_PERIOD);
                 const Tile tl = tile_of(args, wk.tile);
@@ -571,13 +751,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool zero_row = false;
             // masked layout: only rows below the expert's count are written; a warp whose 32
             // rows are all valid stores through TMA, one with some invalid rows row by row
-            bool row_valid = true, all_valid = true;
+            bool row_valid = mine, all_valid = mine;
             if constexpr (C::MASKED) {
                 row_valid = row - g * args.max_m < mcount[g];
                 all_valid = __all_sync(0xffffffffu, row_valid);
             }
             if constexpr (C::GROUPED && !C::MASKED) {
-                if (row < args.M) {
+                if (row < args.M && mine) {
                     const int g0 = __ldg(args.m_indices + m0);
                     const int gi = __ldg(args.m_indices + row);
                     zero_row = gi < 0;
@@ -628,6 +808,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     return;
                 }
+                // a block wholly outside D is neither staged nor stored: staging it would reuse the
+                // buffer of the last store issued, which may still be reading it
+                if (m0 + (int)quarter * 32 >= args.M || n0 + c * 32 >= args.N) return;
                 // the store issued from this buffer two blocks ago has finished reading it
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
@@ -641,7 +824,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0 && m0 + (int)quarter * 32 < args.M && n0 + c * 32 < args.N) {
+                if (lane == 0) {
                     tma_store_2d(&tm_d, blk, n0 + c * 32, m0 + (int)quarter * 32);
                     bulk_commit_group();
                 }
@@ -676,125 +859,141 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     bulk_wait_group_all();  // complete in memory, not only read
                     fence_proxy_async_global();
                 }
-                // publish this slice, then wait (bounded) until every slice of these rows has
-                bool ok = true;
+                // Publish this slice, then reduce without ever waiting on a CTA that may not be
+                // resident.  Share j of these 32 rows (rows [32j/S, 32(j+1)/S)) is summed by whoever
+                // claims it first: slice j itself, if it sees every slice published within a short
+                // poll, or the slice that published last, which claims every share still open.  Each
+                // share is reduced exactly once, always summing the slots in slot order, so the bytes
+                // do not depend on who reduced it.
+                const int S = args.splits;
+                const int cidx = (wk.tail * C::CTAS + (int)rank) * 4 + (int)quarter;
+                int* cnt = args.tail_count + cidx;
+                int* claim = args.tail_claim + cidx * S;
+                int state = 0;  // bit 0: every slice published; bit 1: this slice published last
                 if (lane == 0) {
                     __threadfence();
                     griddep_wait();  // the counters were zeroed by the kernel launched before
-                    int* cnt = args.tail_count + (wk.tail * C::CTAS + (int)rank) * 4 + (int)quarter;
-                    atomicAdd(cnt, 1);
-                    const uint64_t t0 = globaltimer_ns();
-                    while (*reinterpret_cast<volatile int*>(cnt) < args.splits) {
-                        if (*abort_flag) {
-                            ok = false;
-                            break;
+                    if (atomicAdd(cnt, 1) == S - 1) {
+                        state = 3;
+                    } else {
+                        const uint64_t t0 = globaltimer_ns();
+                        const uint64_t limit = args.timeout_ns < kTailPollNs ? args.timeout_ns : kTailPollNs;
+                        while (!*abort_flag) {
+                            if (*reinterpret_cast<volatile int*>(cnt) >= S) {
+                                state = 1;
+                                break;
+                            }
+                            if (globaltimer_ns() - t0 > limit) break;
+                            __nanosleep(64);
                         }
-                        if (globaltimer_ns() - t0 > args.timeout_ns) {
-                            latch_status(args.status, kStatusTimeout);
-                            *abort_flag = 1;
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(64);
                     }
                     __threadfence();
+                    fence_proxy_async_global();  // the other slices' stores, acquired above, before the bulk reads
                 }
-                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-                // this slice's share of the 32 rows (32/S of them, S a power of two): gather every
-                // slot's copy of those rows into this warp's (now free) staging area with one
-                // round of bulk copies, then sum the slots in order, round and store
-                const int S = args.splits;
-                const int r0 = wk.slice * (32 / S), nr = 32 / S;
+                state = __shfl_sync(0xffffffffu, state, 0);
                 const int row_bytes = C::BN * 4;
                 const float* wbase = args.ws + (int64_t)wk.tail * S * slot_stride +
                                      (int64_t)((int)rank * C::BM + (int)quarter * 32) * C::BN;
-                if (lane == 0) {
-                    fence_proxy_async_global();  // the other slices' stores, acquired above, before these reads
-                    mbar_arrive_expect_tx(&gather[warp - 2], (uint32_t)(nr * S * row_bytes));
-                    for (int i = 0; i < nr; ++i)
-                        for (int j = 0; j < S; ++j)
-                            bulk_load(stage + (i * S + j) * row_bytes, wbase + j * slot_stride + (int64_t)(r0 + i) * C::BN,
-                                      (uint32_t)row_bytes, &gather[warp - 2]);
-                }
-                if (!warp_wait(&gather[warp - 2], gather_phase, args, abort_flag)) break;
-                gather_phase ^= 1u;
-                if constexpr (C::TRANS_D) {
-                    // element (row, n0 + c) goes to D[n0 + c][row]: lane l sums columns 4l .. 4l + 3 of
-                    // the nr rows (16-byte shared loads) and writes nr consecutive bf16 of each of the
-                    // four rows D[n0 + 4l + e]
-                    const int row0 = m0 + (int)quarter * 32 + r0;
-                    const uint32_t sbase = smem_u32(stage);
-                    for (int c4 = (int)lane * 4; c4 < C::BN; c4 += 128) {
-                        float acc[16][4];
+                const int P = 32 / S;  // rows per gather pass: P rows of all S slots fill the staging area
+                bool ok = true;
+                const int n_claims = (state & 1) ? ((state & 2) ? S : 1) : 0;
+                for (int i = 0; i < n_claims && ok; ++i) {
+                    const int share = (wk.slice + i) % S;
+                    int won = 0;
+                    if (lane == 0) won = atomicCAS(claim + share, 0, 1) == 0;
+                    if (!__shfl_sync(0xffffffffu, won, 0)) continue;
+                    const int r_end = (share + 1) * 32 / S;
+                    for (int rp = share * 32 / S; rp < r_end; rp += P) {
+                        const int nr = r_end - rp < P ? r_end - rp : P;
+                        // the staging area's previous contents have been read by every lane
+                        __syncwarp();
+                        fence_proxy_async_smem();
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&gather[warp - 2], (uint32_t)(nr * S * row_bytes));
+                            for (int r = 0; r < nr; ++r)
+                                for (int j = 0; j < S; ++j)
+                                    bulk_load(stage + (r * S + j) * row_bytes, wbase + j * slot_stride + (int64_t)(rp + r) * C::BN,
+                                              (uint32_t)row_bytes, &gather[warp - 2]);
+                        }
+                        if (!warp_wait(&gather[warp - 2], gather_phase, args, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        gather_phase ^= 1u;
+                        if constexpr (C::TRANS_D) {
+                            // element (row, n0 + c) goes to D[n0 + c][row]: lane l sums columns 4l .. 4l + 3
+                            // of the nr rows (16-byte shared loads) and writes nr consecutive bf16 of each
+                            // of the four rows D[n0 + 4l + e]
+                            const int row0 = m0 + (int)quarter * 32 + rp;
+                            const uint32_t sbase = smem_u32(stage);
+                            for (int c4 = (int)lane * 4; c4 < C::BN; c4 += 128) {
+                                float acc[16][4];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-                            if (i < nr)
-                                for (int j = 0; j < S; ++j) {
-                                    const float4 x = ld_shared_f32x4(sbase + (uint32_t)((i * S + j) * row_bytes + c4 * 4));
-                                    acc[i][0] += x.x, acc[i][1] += x.y, acc[i][2] += x.z, acc[i][3] += x.w;
+                                for (int r = 0; r < 16; ++r) {
+                                    acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+                                    if (r < nr)
+                                        for (int j = 0; j < S; ++j) {
+                                            const float4 x = ld_shared_f32x4(sbase + (uint32_t)((r * S + j) * row_bytes + c4 * 4));
+                                            acc[r][0] += x.x, acc[r][1] += x.y, acc[r][2] += x.z, acc[r][3] += x.w;
+                                        }
                                 }
-                        }
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int d_row = n0 + c4 + e;
-                            if (d_row >= args.N) continue;
-                            uint32_t packed[8];
+                                for (int e = 0; e < 4; ++e) {
+                                    const int d_row = n0 + c4 + e;
+                                    if (d_row >= args.N) continue;
+                                    uint32_t packed[8];
 #pragma unroll
-                            for (int i2 = 0; i2 < 8; ++i2) {
-                                __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(acc[2 * i2][e], acc[2 * i2 + 1][e]));
-                                packed[i2] = *reinterpret_cast<uint32_t*>(&b2);
-                            }
-                            __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
-                            if (row0 + nr <= args.M) {
-                                // nr is 16, 8, 4 or 2 rows: 32, 16, 8 or 4 aligned bytes
-                                if (nr == 16) {
-                                    reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                                    reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                                } else if (nr == 8) {
-                                    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                                } else if (nr == 4) {
-                                    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-                                } else {
-                                    *reinterpret_cast<uint32_t*>(dst) = packed[0];
+                                    for (int r2 = 0; r2 < 8; ++r2) {
+                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(acc[2 * r2][e], acc[2 * r2 + 1][e]));
+                                        packed[r2] = *reinterpret_cast<uint32_t*>(&b2);
+                                    }
+                                    __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
+                                    const bool aligned = (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
+                                    if (aligned && nr == 16 && row0 + 16 <= args.M) {
+                                        reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                                        reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                                    } else if (aligned && nr == 8 && row0 + 8 <= args.M) {
+                                        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                                    } else {
+#pragma unroll
+                                        for (int r = 0; r < 16; ++r)
+                                            if (r < nr && row0 + r < args.M)
+                                                *reinterpret_cast<uint16_t*>(dst + r) = (uint16_t)(packed[r >> 1] >> (16 * (r & 1)));
+                                    }
                                 }
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 16; ++i)
-                                    if (i < nr && row0 + i < args.M)
-                                        *reinterpret_cast<uint16_t*>(dst + i) = (uint16_t)(packed[i >> 1] >> (16 * (i & 1)));
                             }
-                        }
-                    }
-                } else {
-                    const int col = (int)lane * 8;  // 8 columns per lane
-                    const int n = n0 + col;
-                    for (int i = 0; i < nr; ++i) {
-                        const int row = m0 + (int)quarter * 32 + r0 + i;
-                        if (row >= args.M || col >= C::BN || n >= args.N) continue;
-                        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        for (int j = 0; j < S; ++j) {
-                            const uint32_t a4 = smem_u32(stage) + (uint32_t)((i * S + j) * row_bytes + col * 4);
-                            const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
-                            v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
-                            v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-                        }
-                        __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
-                        if (n + 8 <= args.N) {
-                            uint32_t o[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(v[2 * e], v[2 * e + 1]));
-                                o[e] = *reinterpret_cast<uint32_t*>(&b2);
-                            }
-                            *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
                         } else {
+                            const int col = (int)lane * 8;  // 8 columns per lane
+                            const int n = n0 + col;
+                            for (int r = 0; r < nr; ++r) {
+                                const int row = m0 + (int)quarter * 32 + rp + r;
+                                if (row >= args.M || col >= C::BN || n >= args.N) continue;
+                                float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                                for (int j = 0; j < S; ++j) {
+                                    const uint32_t a4 = smem_u32(stage) + (uint32_t)((r * S + j) * row_bytes + col * 4);
+                                    const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
+                                    v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
+                                    v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
+                                }
+                                __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
+                                if (n + 8 <= args.N) {
+                                    uint32_t o[4];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (n + e < args.N) dst[e] = __float2bfloat16_rn(v[e]);
+                                    for (int e = 0; e < 4; ++e) {
+                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(v[2 * e], v[2 * e + 1]));
+                                        o[e] = *reinterpret_cast<uint32_t*>(&b2);
+                                    }
+                                    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e)
+                                        if (n + e < args.N) dst[e] = __float2bfloat16_rn(v[e]);
+                                }
+                            }
                         }
                     }
                 }
+                if (!ok) break;
             } else if constexpr (C::ACC_BUFS == 2) {
 #pragma unroll 1
                 for (int c = 0; c < C::BN / 32; ++c) {

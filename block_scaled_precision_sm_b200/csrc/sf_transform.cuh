@@ -3,65 +3,186 @@
 // para Huawei Ascend 950", section "Qué incluye el lanzamiento": each pair of UE8M0
 // factors along K in one 16-bit integer, MN-major).
 //
-// One CTA transposes a 64-row x 64-block tile through shared memory: the reads run along
-// K (the input's contiguous axis), the writes along MN (the output's contiguous axis),
-// so both sides are coalesced.  The transform moves a few bytes per scale and is bound
-// by DRAM bandwidth.
+// One CTA turns a tile of 128 rows x 64 scale blocks around through shared memory.  Reads run
+// along K (the input's contiguous axis) in VEC-byte vectors, as wide as the input's row stride
+// and base alignment allow, with every lane busy whatever kb is (the tile's (row, vector) pairs
+// are numbered linearly); the exponent bytes land transposed in shared memory, K-major, so that
+// each output store is one 16-byte run of eight MN-consecutive words, built from two 8-byte
+// shared loads with byte permutes.  The transform moves a few bytes per scale and is bound by
+// DRAM bandwidth; each thread issues all of its loads before it uses any.
 #pragma once
+
+#include <cuda_runtime.h>
 
 #include <cstdint>
 
 namespace bsp {
 
-constexpr int kSfTileMN = 64;
-constexpr int kSfTileKB = 64;
+constexpr int kSfTileMN = 128;  // rows per CTA
+constexpr int kSfTileKB = 64;   // scale blocks per CTA
+constexpr int kSfThreads = 256;
+
+template <int VEC>
+struct SfVec;
+template <>
+struct SfVec<16> {
+    using T = uint4;
+    static __device__ __forceinline__ uint32_t word(const T& v, int i) {
+        return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+    }
+};
+template <>
+struct SfVec<8> {
+    using T = uint2;
+    static __device__ __forceinline__ uint32_t word(const T& v, int i) { return i == 0 ? v.x : v.y; }
+};
+template <>
+struct SfVec<4> {
+    using T = uint32_t;
+    static __device__ __forceinline__ uint32_t word(const T& v, int) { return v; }
+};
+template <>
+struct SfVec<1> {
+    using T = uint8_t;
+    static __device__ __forceinline__ uint32_t word(const T& v, int) { return v; }
+};
 
 // IN_KIND 0: fp32 power-of-two scales (UE8M0 byte = biased fp32 exponent);
-// IN_KIND 1: uint8 UE8M0 bytes.
-template <int IN_KIND>
-__global__ void __launch_bounds__(256) sf_transform_kernel(const void* __restrict__ in, int mn, int kb,
-                                                           int64_t ld_in, uint16_t* __restrict__ out,
-                                                           int64_t ld_out, int* status) {
-    __shared__ uint8_t e[kSfTileMN][kSfTileKB + 4];
+// IN_KIND 1: uint8 UE8M0 bytes.  VEC: bytes per global load (16, 8 or 4 for fp32; 16, 8, 4 or
+// 1 for bytes); the row stride ld_in and the base are multiples of VEC bytes.
+template <int IN_KIND, int VEC>
+__global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __restrict__ in, int mn, int kb,
+                                                                  int64_t ld_in, uint16_t* __restrict__ out,
+                                                                  int64_t ld_out, int* status) {
+    constexpr int ES = IN_KIND == 0 ? 4 : 1;       // input element bytes
+    constexpr int EV = VEC / ES;                   // elements per load
+    static_assert(EV >= 1 && kSfTileKB % EV == 0, "vector width");
+    constexpr int MAX_VECS = kSfTileMN * (kSfTileKB / EV) / kSfThreads;  // loads per thread, at most
+    constexpr int PITCH = kSfTileMN + 16;          // bytes per K block in shared memory
+    using V = typename SfVec<VEC>::T;
+    __shared__ __align__(16) uint8_t eT[kSfTileKB][PITCH];
+
     const int r0 = blockIdx.x * kSfTileMN;
     const int k0 = blockIdx.y * kSfTileKB;
-    const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+    const int kn = min(kSfTileKB, kb - k0);         // scale blocks in this tile
+    const int rn = min(kSfTileMN, mn - r0);         // input rows in this tile (<= 0: padding only)
+    const int vpr = (kn + EV - 1) / EV;             // loads per row
+    const int total = rn > 0 ? rn * vpr : 0;
+    const int t = threadIdx.x;
     bool bad = false;
+
+    // all loads first (up to MAX_VECS in flight per thread), then the bytes into shared memory
+    V v[MAX_VECS];
 #pragma unroll
-    for (int i = ty; i < kSfTileMN; i += 8) {
-        const int r = r0 + i;
+    for (int it = 0; it < MAX_VECS; ++it) {
+        const int idx = t + it * kSfThreads;
+        if (idx < total) {
+            const int i = idx / vpr, k = (idx - i * vpr) * EV;
+            const char* src = static_cast<const char*>(in) + ((int64_t)(r0 + i) * ld_in + k0 + k) * ES;
+            if (k + EV <= kn) {
+                v[it] = __ldg(reinterpret_cast<const V*>(src));
+            } else {  // a partial vector at the end of a row: the elements that exist, zeros after
+                uint32_t w[VEC >= 4 ? VEC / 4 : 1] = {};
 #pragma unroll
-        for (int j = tx; j < kSfTileKB; j += 32) {
-            const int k = k0 + j;
-            uint32_t v = 0;
-            if (r < mn && k < kb) {
-                if constexpr (IN_KIND == 0) {
-                    const uint32_t bits = __float_as_uint(__ldg(static_cast<const float*>(in) + (int64_t)r * ld_in + k));
-                    v = (bits >> 23) & 0xFFu;
-                    // exact positive normal power of two: sign 0, mantissa 0, exponent 1..254
-                    bad |= (bits & 0x807FFFFFu) != 0u || v == 0u || v == 255u;
-                } else {
-                    v = __ldg(static_cast<const uint8_t*>(in) + (int64_t)r * ld_in + k);
+                for (int e = 0; e < EV; ++e) {
+                    if (k + e < kn) {
+                        const uint32_t x = ES == 4 ? __ldg(reinterpret_cast<const uint32_t*>(src) + e)
+                                                   : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(src) + e);
+                        if (ES == 4)
+                            w[e] = x;
+                        else
+                            w[e / 4] |= x << (8 * (e % 4));
+                    }
+                }
+                if constexpr (VEC == 16)
+                    v[it] = make_uint4(w[0], w[1], w[2], w[3]);
+                else if constexpr (VEC == 8)
+                    v[it] = make_uint2(w[0], w[1]);
+                else if constexpr (VEC == 4)
+                    v[it] = w[0];
+                else
+                    v[it] = (uint8_t)w[0];
+            }
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < MAX_VECS; ++it) {
+        const int idx = t + it * kSfThreads;
+        if (idx < total) {
+            const int i = idx / vpr, k = (idx - i * vpr) * EV;
+#pragma unroll
+            for (int e = 0; e < EV; ++e) {
+                if (k + e < kn) {
+                    uint32_t b;
+                    if constexpr (IN_KIND == 0) {
+                        const uint32_t bits = SfVec<VEC>::word(v[it], e);
+                        b = (bits >> 23) & 0xFFu;
+                        // an exact positive normal power of two: sign 0, mantissa 0, exponent 1..254
+                        bad |= (bits & 0x807FFFFFu) != 0u || b == 0u || b == 255u;
+                    } else {
+                        b = (SfVec<VEC>::word(v[it], e / 4) >> (8 * (e % 4))) & 0xFFu;
+                        bad |= b == 255u;  // UE8M0 0xFF is NaN
+                    }
+                    eT[k + e][i] = (uint8_t)b;
                 }
             }
-            e[i][j] = static_cast<uint8_t>(v);
         }
     }
     __syncthreads();
-    const int words = (kb + 1) / 2;
-#pragma unroll
-    for (int w = ty; w < kSfTileKB / 2; w += 8) {
-        const int jw = k0 / 2 + w;
-        if (jw >= words) break;
-#pragma unroll
-        for (int i = tx; i < kSfTileMN; i += 32) {
-            const int r = r0 + i;
-            if (r < ld_out)
-                out[(int64_t)jw * ld_out + r] =
-                    static_cast<uint16_t>(e[i][2 * w] | (static_cast<uint32_t>(e[i][2 * w + 1]) << 8));
-        }
+
+    // words (k0/2 + j) for rows r0 + 8g .. r0 + 8g + 7: rows past mn and the high byte past an
+    // odd kb are 0; rows past ld_out are not written (ld_out is a multiple of 8)
+    const int wn = (kn + 1) / 2;
+    for (int idx = t; idx < wn * (kSfTileMN / 8); idx += kSfThreads) {
+        const int j = idx / (kSfTileMN / 8), g = idx - j * (kSfTileMN / 8);
+        const int r = r0 + 8 * g;
+        if (r >= ld_out) continue;
+        const int valid = mn - r;  // rows of this run that hold scales
+        const uint64_t keep = valid >= 8 ? ~0ull : valid <= 0 ? 0ull : (1ull << (8 * valid)) - 1ull;
+        const uint64_t lo = *reinterpret_cast<const uint64_t*>(&eT[2 * j][8 * g]) & keep;
+        const uint64_t hi = 2 * j + 1 < kn ? *reinterpret_cast<const uint64_t*>(&eT[2 * j + 1][8 * g]) & keep : 0ull;
+        const uint32_t l0 = (uint32_t)lo, l1 = (uint32_t)(lo >> 32), h0 = (uint32_t)hi, h1 = (uint32_t)(hi >> 32);
+        // word of row q = byte q of lo | byte q of hi << 8
+        *reinterpret_cast<uint4*>(out + (int64_t)(k0 / 2 + j) * ld_out + r) =
+            make_uint4(__byte_perm(l0, h0, 0x5140), __byte_perm(l0, h0, 0x7362), __byte_perm(l1, h1, 0x5140),
+                       __byte_perm(l1, h1, 0x7362));
     }
-    if (IN_KIND == 0 && __any_sync(0xffffffffu, bad) && tx == 0) atomicCAS(status, 0, -7);
+    if (__any_sync(0xffffffffu, bad) && (t % 32) == 0) atomicCAS(status, 0, -7);
+}
+
+// Widest load (bytes) that the input's base address and row stride allow.
+inline int sf_transform_vec(const void* in, int in_kind, int64_t ld_in) {
+    const int es = in_kind == 0 ? 4 : 1;
+    const uint64_t a = reinterpret_cast<uintptr_t>(in) | (uint64_t)(ld_in * es);
+    for (int v : {16, 8, 4})
+        if (a % (uint64_t)v == 0) return v;
+    return es == 4 ? 4 : 1;
+}
+
+// Launch on `stream`; false if the launch failed or the grid is too large.
+inline bool launch_sf_transform(const void* in, int in_kind, int mn, int kb, int64_t ld_in, uint16_t* out,
+                                int64_t ld_out, int* status, cudaStream_t stream) {
+    const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
+    if (grid.y > 65535u) return false;
+    const int vec = sf_transform_vec(in, in_kind, ld_in);
+    if (in_kind == 0) {
+        if (vec == 16)
+            sf_transform_kernel<0, 16><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+        else if (vec == 8)
+            sf_transform_kernel<0, 8><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+        else
+            sf_transform_kernel<0, 4><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+    } else {
+        if (vec == 16)
+            sf_transform_kernel<1, 16><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+        else if (vec == 8)
+            sf_transform_kernel<1, 8><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+        else if (vec == 4)
+            sf_transform_kernel<1, 4><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+        else
+            sf_transform_kernel<1, 1><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
+    }
+    return cudaGetLastError() == cudaSuccess;
 }
 
 }  // namespace bsp

@@ -34,6 +34,9 @@
  *     device, and free it on the same stream.  Every call can be captured in a CUDA graph;
  *     under capture the scratch becomes a graph memory node.
  *   - Results are deterministic: the same inputs give the same bytes on every run.
+ *   - The GEMMs bring their operand tiles into L2 a few K steps ahead of loading them; the
+ *     environment variable BSP_L2_PREFETCH_KSTEPS (read once per process, 0..64, 0 = off)
+ *     sets how many.  It changes timing only, never results.
  *
  * Packed scale-factor layout ("SF words"): for a matrix with MN scale rows and KB scale
  * blocks along K, the SF tensor is int16 [ceil(KB/2)][ld], with
@@ -149,7 +152,8 @@ int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, 
  *   in_kind 0: fp32 scales, each an exact positive normal power of two; its biased
  *              exponent (bits 30..23) is the UE8M0 byte.  A value that is not such a
  *              power of two latches BSP_ERR_DEVICE_CHECK (its byte is still written).
- *   in_kind 1: uint8 biased UE8M0 bytes, copied as they are.
+ *   in_kind 1: uint8 biased UE8M0 bytes, copied as they are; the byte 0xFF (NaN in UE8M0)
+ *              latches BSP_ERR_DEVICE_CHECK (it is still written).
  *   ld_out >= mn and ld_out*2 a multiple of 16 bytes; sf_out must not overlap sf_in.
  * The caller decides whether a tensor is already packed ("reuse or convert",
  * "Fatores de escala FP8 e o formato UE8M0 no Ascend"); this call always converts.
@@ -209,8 +213,10 @@ int quantize_fp8_ue8m0(const void* x, int in_kind, int rows, int cols, int64_t l
  * Every call shares the one scratch array and overwrites it: calls that overlap on the GPU
  * (different streams, or different host threads on one device) race on it and must be
  * ordered by the caller.  The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before any stream
- * capture.
+ * (cudaGetSymbolAddress) with that device current and keeps it for the process; make that
+ * first call before any stream capture, and do not use this entry point on a device after
+ * cudaDeviceReset, or from a context other than the device's primary one (the kept address
+ * would then be stale).  A scale byte 0xFF (NaN) latches BSP_ERR_DEVICE_CHECK in `status`.
  */
 int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const void* B, const void* sfb_e8m0, void* D,
                         int* status, int M, int N, int K, int64_t lda, int64_t ldb, int64_t ldd,

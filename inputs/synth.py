@@ -187,8 +187,9 @@ def dirichlet_segments(rng: np.random.Generator, groups: int, total_rows: int, a
 
 
 def grouped_fp8_problem(groups: int, total_rows: int, n: int, k: int, seed: int = 0,
-                        alpha: float = 1.0, align: int = 128, counts=None):
-    """M-grouped contiguous FP8 problem (MoE): expert segments padded to `align` rows."""
+                        alpha: float = 1.0, align: int = 128, counts=None, b_block_rows: int = 128):
+    """M-grouped contiguous FP8 problem (MoE): expert segments padded to `align` rows; each
+    expert's B has b_block_rows x 128 scale blocks (128 by default, 1 = one scale per row)."""
     rng = np.random.default_rng(seed)
     if counts is None:
         counts = dirichlet_segments(rng, groups, total_rows, alpha)
@@ -209,17 +210,24 @@ def grouped_fp8_problem(groups: int, total_rows: int, n: int, k: int, seed: int 
         src += c
         dst += int(padded[g])
     del a_codes, a_sf
-    b = np.empty((groups, n, k), np.uint8)
-    sfb = np.empty((groups, -(-n // 128), k // 128), np.uint8)
-    for g in range(groups):
-        b[g], sfb[g] = _fp8_operand(n, k, seed + 2 + g, 128)
+    b, sfb = _expert_weights(groups, n, k, seed, b_block_rows)
     return {"kind": "grouped_fp8", "G": groups, "M": m_total, "N": n, "K": k, "A": a, "sfa": sfa,
-            "B": b, "sfb": sfb, "m_indices": m_indices, "counts": counts, "gran_n": 128}
+            "B": b, "sfb": sfb, "m_indices": m_indices, "counts": counts, "gran_n": b_block_rows}
 
 
-def masked_fp8_problem(groups: int, max_m: int, n: int, k: int, seed: int = 0, counts=None):
+def _expert_weights(groups: int, n: int, k: int, seed: int, b_block_rows: int):
+    """Per-expert B [G, N, K] and its UE8M0 exponents [G, ceil(N/b_block_rows), K/128]."""
+    b = np.empty((groups, n, k), np.uint8)
+    sfb = np.empty((groups, -(-n // b_block_rows), k // 128), np.uint8)
+    for g in range(groups):
+        b[g], sfb[g] = _fp8_operand(n, k, seed + 2 + g, b_block_rows)
+    return b, sfb
+
+
+def masked_fp8_problem(groups: int, max_m: int, n: int, k: int, seed: int = 0, counts=None,
+                       b_block_rows: int = 128):
     """Masked grouped FP8 problem: A [G, max_m, K] (1x128 scales, [G*max_m, K/128]),
-    B [G, N, K] (128x128 scales), masked_m [G] valid rows per expert."""
+    B [G, N, K] (b_block_rows x 128 scales, 128 by default), masked_m [G] valid rows per expert."""
     rng = np.random.default_rng(seed)
     if counts is None:
         counts = rng.integers(0, max_m + 1, size=groups)
@@ -227,10 +235,7 @@ def masked_fp8_problem(groups: int, max_m: int, n: int, k: int, seed: int = 0, c
     if masked_m.shape != (groups,) or masked_m.min() < 0 or masked_m.max() > max_m:
         raise ValueError("counts must be G values in [0, max_m]")
     a, sfa = _fp8_operand(groups * max_m, k, seed + 1, 1)
-    b = np.empty((groups, n, k), np.uint8)
-    sfb = np.empty((groups, -(-n // 128), k // 128), np.uint8)
-    for g in range(groups):
-        b[g], sfb[g] = _fp8_operand(n, k, seed + 2 + g, 128)
+    b, sfb = _expert_weights(groups, n, k, seed, b_block_rows)
     return {"kind": "masked_fp8", "G": groups, "max_m": max_m, "N": n, "K": k,
             "A": a.reshape(groups, max_m, k), "sfa": sfa, "B": b, "sfb": sfb, "masked_m": masked_m,
-            "gran_n": 128}
+            "gran_n": b_block_rows}

@@ -57,12 +57,42 @@ def test_transform_bit_exact_fp32(ops, orc, mn, kb):
     assert np.array_equal(got.cpu().numpy(), orc.sf_pack(orc.fp32_scales_to_ue8m0(s), ld_out=ld))
 
 
+# The transform loads along K as wide as the input's row stride allows (16, 8, 4 or 1 bytes):
+# every width, a vector cut short at the end of a row, several K tiles and a padded ld_out.
+@pytest.mark.parametrize("kind,mn,kb,ld_in", [("u8", 300, 64, 64), ("u8", 257, 56, 56), ("u8", 130, 40, 48),
+                                              ("u8", 99, 20, 20), ("u8", 64, 130, 130), ("fp32", 200, 6, 8),
+                                              ("fp32", 333, 5, 6), ("fp32", 77, 3, 3), ("fp32", 1000, 150, 152)])
+def test_transform_vector_widths(ops, orc, kind, mn, kb, ld_in):
+    rng = np.random.default_rng(mn * kb)
+    e = rng.integers(1, 255, size=(mn, kb), dtype=np.uint8)
+    full = np.zeros((mn, ld_in), np.uint8 if kind == "u8" else np.float32)
+    if kind == "u8":
+        full[:, :kb] = e
+    else:
+        full[:, :kb] = np.ldexp(np.float32(1.0), e.astype(np.int32) - 127)
+    src = to_dev(full)[:, :kb]
+    ld_out = (mn + 7) // 8 * 8 + 8
+    got = ops.transform_sf_ue8m0(src, ld_out=ld_out)
+    _status_ok(ops)
+    assert np.array_equal(got.cpu().numpy(), orc.sf_pack(e, ld_out=ld_out))
+
+
 def test_transform_flags_bad_scale(ops):
     s = np.ones((16, 4), np.float32)
     s[3, 2] = 3.0
     ops.transform_sf_ue8m0(to_dev(s))
     assert ops.device_status() == -7
     _status_ok(ops)  # cleared
+
+
+def test_transform_flags_nan_byte(ops, orc):
+    # UE8M0 0xFF is NaN: the uint8 path latches the check too, and still packs the byte
+    e = np.full((40, 6), 127, np.uint8)
+    e[21, 5] = 0xFF
+    got = ops.transform_sf_ue8m0(to_dev(e))
+    assert ops.device_status() == -7
+    _status_ok(ops)  # cleared
+    assert np.array_equal(got.cpu().numpy(), orc.sf_pack(e, ld_out=got.shape[1]))
 
 
 def test_reuse_or_convert(ops):
@@ -263,6 +293,43 @@ def test_split_last_wave_sampled(ops, orc, kind, m, n, k):
     check_gemm(got, ref(orc), f"{kind} last wave {m}x{n}x{k} {plan}")
 
 
+# Slice counts that are not powers of two: the rows of each epilogue warp are cut into shares
+# of different sizes, some needing two gather passes, and in the transposed kernel the shares
+# start at unaligned positions of D's rows.
+@pytest.mark.parametrize("kind,m,n,k,gran,splits", [("fp8", 512, 2560, 3072, 128, 3), ("fp8", 96, 3584, 5120, 1, 5),
+                                                    ("bf16", 64, 1792, 6144, 1, 10),
+                                                    ("fp4", 256, 2560, 16384, 1, 7)])
+def test_split_any_slice_count(ops, orc, kind, m, n, k, gran, splits):
+    plan = ops.gemm_plan(kind, m, n, k)
+    assert plan["splits"] == splits, plan
+    rng = np.random.default_rng(n)
+    rows = np.arange(m, dtype=np.int32)  # every row: every share of every warp
+    cols = np.unique(np.concatenate([rng.integers(c, min(c + 128, n), 5) for c in range(0, n, 128)])).astype(np.int32)
+    if m * n * k <= 2 ** 33:
+        rows, cols = None, None
+    got, ref = _run_kind(ops, kind, m, n, k, seed=m + n, gran=gran, rows=rows, cols=cols)
+    check_gemm(got, ref(orc), f"{kind} {splits} slices {m}x{n}x{k} {plan}")
+
+
+def test_split_tails_on_two_concurrent_streams(ops, orc):
+    # two split-tail GEMMs enqueued on two streams at once: neither waits on a CTA of the other,
+    # and a slice never waits on an unscheduled slice of its own tile
+    probs = [inputs.dense_fp8_problem(256, 1024, 4096, seed=s) for s in (41, 42)]
+    assert ops.gemm_plan("fp8", 256, 1024, 4096)["splits"] > 1
+    devs = [[to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")] for p in probs]
+    outs = [torch.empty((256, 1024), dtype=torch.bfloat16, device="cuda") for _ in probs]
+    streams = [torch.cuda.Stream() for _ in probs]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for d, o, st in zip(devs, outs, streams):
+            with torch.cuda.stream(st):
+                ops.gemm_fp8_nt(*d, o)
+    torch.cuda.synchronize()
+    _status_ok(ops)
+    for p, o in zip(probs, outs):
+        check_gemm(bf16_to_f64(o), orc.gemm_fp8(p["A"], p["sfa"], p["B"], p["sfb"]), "concurrent split")
+
+
 def test_split_is_deterministic(ops):
     # slices are added in a fixed order, so repeated runs give identical bytes
     p = inputs.dense_fp8_problem(256, 1024, 4096, seed=5)
@@ -315,6 +382,37 @@ def test_grouped(ops, orc, counts, n, k):
     check_gemm(got, ref, "grouped")
     pad = p["m_indices"] < 0
     assert np.all(got[pad] == 0.0)  # padding rows are exactly zero
+
+
+def test_grouped_pair_tiles_odd_and_even_runs(ops, orc):
+    # experts with 1, 2, 3, 1, 2, 0 and 5 blocks of 128 rows: pairs of blocks of one expert run on
+    # CTA pairs, an odd last block alone (its peer CTA's rows, the next expert's, are not written)
+    counts = [100, 256, 300, 1, 129, 0, 600]
+    p = inputs.grouped_fp8_problem(len(counts), sum(counts), 448, 512, seed=23, counts=counts)
+    plan = ops.gemm_plan("grouped_fp8", p["M"], 448, 512)
+    assert plan["tile_m"] == 256 and plan["tile_n"] == 224, plan
+    D = _grouped(ops, p)
+    _status_ok(ops)
+    got = bf16_to_f64(D)
+    check_gemm(got, orc.gemm_grouped_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["m_indices"]), "grouped pair tiles")
+    assert np.all(got[p["m_indices"] < 0] == 0.0)
+
+
+def test_grouped_beyond_the_pair_list_runs_single_cta(ops, orc):
+    # more than 2048 blocks of 128 rows: the single-CTA grouped kernel (128 x 224 tiles)
+    counts = [2048 * 128 - 50, 128 + 50, 70]
+    n, k = 64, 128
+    p = inputs.grouped_fp8_problem(3, sum(counts), n, k, seed=29, counts=counts)
+    assert p["M"] // 128 > 2048
+    assert ops.gemm_plan("grouped_fp8", p["M"], n, k)["tile_m"] == 128
+    D = _grouped(ops, p)
+    _status_ok(ops)
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([rng.choice(p["M"], 300, replace=False),
+                                     np.arange(p["M"] - 400, p["M"])])).astype(np.int32)
+    got = bf16_to_f64(D[torch.from_numpy(rows).long().cuda()])
+    ref = orc.gemm_grouped_fp8(p["A"], p["sfa"], p["B"], p["sfb"], p["m_indices"], rows=rows)
+    check_gemm(got, ref, "grouped, single-CTA tiles")
 
 
 def test_grouped_padding_rows_zero_whatever_a_holds(ops, orc):
