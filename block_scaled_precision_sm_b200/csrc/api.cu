@@ -39,7 +39,7 @@ std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 
 // K steps the GEMMs' L2 prefetch of operand tiles runs ahead of their loads; the environment
 // variable BSP_L2_PREFETCH_KSTEPS, read once, overrides it (0 turns the prefetch off).
-constexpr int kDefaultPrefetchKSteps = 8;
+constexpr int kDefaultPrefetchKSteps = 0;
 int prefetch_ksteps() {
     static const int v = [] {
         const char* e = std::getenv("BSP_L2_PREFETCH_KSTEPS");

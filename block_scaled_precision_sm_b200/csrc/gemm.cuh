@@ -920,61 +920,69 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             break;
                         }
                         gather_phase ^= 1u;
-                        if constexpr (C::TRANS_D) {
-                            // element (row, n0 + c) goes to D[n0 + c][row]: lane l sums columns 4l .. 4l + 3
-                            // of the nr rows (16-byte shared loads) and writes nr consecutive bf16 of each
-                            // of the four rows D[n0 + 4l + e]
-                            const int row0 = m0 + (int)quarter * 32 + rp;
-                            const uint32_t sbase = smem_u32(stage);
-                            for (int c4 = (int)lane * 4; c4 < C::BN; c4 += 128) {
-                                float acc[16][4];
-#pragma unroll
-                                for (int r = 0; r < 16; ++r) {
-                                    acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
-                                    if (r < nr)
-                                        for (int j = 0; j < S; ++j) {
-                                            const float4 x = ld_shared_f32x4(sbase + (uint32_t)((r * S + j) * row_bytes + c4 * 4));
-                                            acc[r][0] += x.x, acc[r][1] += x.y, acc[r][2] += x.z, acc[r][3] += x.w;
-                                        }
+                        // The reduction runs once, at the end of the kernel, so its instructions are
+                        // cold: compact loops, not unrolled bodies.  First every row's S copies are
+                        // added, in slot order, into its slot-0 copy (16 bytes per lane, consecutive
+                        // lanes on consecutive bytes); then the sums are rounded and written.
+                        const uint32_t sbase = smem_u32(stage);
+                        const uint32_t row_pitch = (uint32_t)(S * row_bytes);  // between gathered rows
+#pragma unroll 1
+                        for (int r = 0; r < nr; ++r) {
+#pragma unroll 1
+                            for (int c = (int)lane * 4; c < C::BN; c += 128) {
+                                const uint32_t a0 = sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u;
+                                float4 acc = ld_shared_f32x4(a0);
+#pragma unroll 1
+                                for (int j = 1; j < S; ++j) {
+                                    const float4 x = ld_shared_f32x4(a0 + (uint32_t)(j * row_bytes));
+                                    acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
                                 }
+                                st_shared_f32x4(a0, acc);
+                            }
+                        }
+                        __syncwarp();
+                        if constexpr (C::TRANS_D) {
+                            // element (row, n0 + c) goes to D[n0 + c][row]: lane l writes D rows n0 + l,
+                            // n0 + l + 32, ..., each with the nr consecutive bf16 of its column, eight at
+                            // a time (one 16-byte store where D's row allows it)
+                            const int row0 = m0 + (int)quarter * 32 + rp;
+#pragma unroll 1
+                            for (int c = (int)lane; c < C::BN; c += 32) {
+                                const int d_row = n0 + c;
+                                if (d_row >= args.N) continue;
+                                __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
+#pragma unroll 1
+                                for (int r8 = 0; r8 < nr; r8 += 8) {
+                                    uint32_t w[4];
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int d_row = n0 + c4 + e;
-                                    if (d_row >= args.N) continue;
-                                    uint32_t packed[8];
-#pragma unroll
-                                    for (int r2 = 0; r2 < 8; ++r2) {
-                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(acc[2 * r2][e], acc[2 * r2 + 1][e]));
-                                        packed[r2] = *reinterpret_cast<uint32_t*>(&b2);
+                                    for (int h = 0; h < 4; ++h) {
+                                        const int r = r8 + 2 * h;
+                                        const float lo = r < nr ? ld_shared_f32(sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u) : 0.f;
+                                        const float hi = r + 1 < nr ? ld_shared_f32(sbase + (uint32_t)(r + 1) * row_pitch + (uint32_t)c * 4u) : 0.f;
+                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(lo, hi));
+                                        w[h] = *reinterpret_cast<uint32_t*>(&b2);
                                     }
-                                    __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
-                                    const bool aligned = (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
-                                    if (aligned && nr == 16 && row0 + 16 <= args.M) {
-                                        reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                                        reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                                    } else if (aligned && nr == 8 && row0 + 8 <= args.M) {
-                                        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                                    __nv_bfloat16* d8 = dst + r8;
+                                    if (r8 + 8 <= nr && row0 + r8 + 8 <= args.M && (reinterpret_cast<uintptr_t>(d8) & 15u) == 0) {
+                                        *reinterpret_cast<uint4*>(d8) = make_uint4(w[0], w[1], w[2], w[3]);
                                     } else {
 #pragma unroll
-                                        for (int r = 0; r < 16; ++r)
-                                            if (r < nr && row0 + r < args.M)
-                                                *reinterpret_cast<uint16_t*>(dst + r) = (uint16_t)(packed[r >> 1] >> (16 * (r & 1)));
+                                        for (int r = 0; r < 8; ++r)
+                                            if (r8 + r < nr && row0 + r8 + r < args.M)
+                                                *reinterpret_cast<uint16_t*>(d8 + r) = (uint16_t)(w[r >> 1] >> (16 * (r & 1)));
                                     }
                                 }
                             }
                         } else {
                             const int col = (int)lane * 8;  // 8 columns per lane
                             const int n = n0 + col;
+#pragma unroll 1
                             for (int r = 0; r < nr; ++r) {
                                 const int row = m0 + (int)quarter * 32 + rp + r;
                                 if (row >= args.M || col >= C::BN || n >= args.N) continue;
-                                float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                                for (int j = 0; j < S; ++j) {
-                                    const uint32_t a4 = smem_u32(stage) + (uint32_t)((r * S + j) * row_bytes + col * 4);
-                                    const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
-                                    v[0] += x0.x, v[1] += x0.y, v[2] += x0.z, v[3] += x0.w;
-                                    v[4] += x1.x, v[5] += x1.y, v[6] += x1.z, v[7] += x1.w;
-                                }
+                                const uint32_t a4 = sbase + (uint32_t)r * row_pitch + (uint32_t)col * 4u;
+                                const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
+                                const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                                 __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
                                 if (n + 8 <= args.N) {
                                     uint32_t o[4];

@@ -190,6 +190,17 @@ __device__ __forceinline__ float4 ld_shared_f32x4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void st_shared_f32x4(uint32_t addr, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // Contiguous global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
 // aligned), completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
