@@ -5,7 +5,6 @@
 
 #include <atomic>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -37,17 +36,6 @@ std::mutex g_mu;
 DeviceCtx g_dev[kMaxDevices];
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 
-// K steps the GEMMs' L2 prefetch of operand tiles runs ahead of their loads; the environment
-// variable BSP_L2_PREFETCH_KSTEPS, read once, overrides it (0 turns the prefetch off).
-constexpr int kDefaultPrefetchKSteps = 0;
-int prefetch_ksteps() {
-    static const int v = [] {
-        const char* e = std::getenv("BSP_L2_PREFETCH_KSTEPS");
-        const int x = e ? std::atoi(e) : kDefaultPrefetchKSteps;
-        return x < 0 ? 0 : (x > 64 ? 64 : x);
-    }();
-    return v;
-}
 std::atomic<uint64_t> g_launches{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -223,7 +211,6 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     a.group_m = 16;
     a.status = ctx.status;
     a.timeout_ns = g_timeout_ns.load();
-    a.prefetch = prefetch_ksteps();
     const int workers = a.num_work < max_workers ? a.num_work : max_workers;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -385,16 +372,15 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, pools[dev], stream) == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
 }
 
-// Chunk tensor map: 8-byte elements, one chunk per (row tile, group [, expert]); a box is the
-// chunks of `batch` consecutive groups of one row tile (groups past the last read as zeros).
-int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int q, int experts_or_neg, int batch) {
+// Chunk tensor map: 8-byte elements, one chunk per (row tile, group [, expert]).
+int chunk_map(CUtensorMap* m, const void* base, int chunk_bytes, int tiles, int q, int experts_or_neg) {
     // experts_or_neg < 0: a rank-4 map over -experts_or_neg experts (the grouped kernel's 4-D loads)
     const int experts = experts_or_neg < 0 ? -experts_or_neg : experts_or_neg;
     const cuuint64_t dims[4] = {(cuuint64_t)(chunk_bytes / 8), (cuuint64_t)tiles, (cuuint64_t)q,
                                 (cuuint64_t)experts};
     const cuuint64_t strides[3] = {(cuuint64_t)chunk_bytes, (cuuint64_t)chunk_bytes * tiles,
                                    (cuuint64_t)chunk_bytes * tiles * q};
-    const cuuint32_t box[4] = {(cuuint32_t)(chunk_bytes / 8), 1, (cuuint32_t)batch, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)(chunk_bytes / 8), 1, 1, 1};
     return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, experts_or_neg < 0 ? 4 : 3, base, dims, strides, box,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
@@ -478,9 +464,8 @@ int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_
         char* wa = base;
         char* wb = wa + ScaleChunks<C>(o, a).a_bytes;
         rc = launch_sf_layout(o.sfa, la, wa, o.sfb, lb, wb, count, tail_bytes ? tail_count_bytes<C>(p) : 0, stream);
-        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1, C::SF_BATCH);
-        if (rc == BSP_OK)
-            rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1, C::SF_BATCH);
+        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1);
+        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1);
     } else {
         tsa = ta, tsb = tb;  // not read
         if (tail_bytes && cudaMemsetAsync(count, 0, (size_t)tail_count_bytes<C>(p), stream) != cudaSuccess)

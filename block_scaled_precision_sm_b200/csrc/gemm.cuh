@@ -7,13 +7,12 @@
 // operandos e pipelining na prática", rebuilt for Blackwell):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) into an S-stage shared-memory
 //               ring ("full"/"empty" mbarriers, transaction-counted); the first stage of every
-//               batch of SF_BATCH scale groups (SF_PERIOD K steps each) also carries the
-//               batch's chunks of scale words into a two-slot scale ring (released by its own
-//               barriers), laid out beforehand (sf_layout.cuh) exactly as the scale copy reads
+//               scale group (SF_PERIOD K steps) also carries one chunk of scale words per
+//               operand, laid out beforehand (sf_layout.cuh) exactly as the scale copy reads
 //               them, so no thread rearranges scales on chip.
-//   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers, issues
-//               one burst of tcgen05.cp per batch (every group's chunks into its own TMEM slot)
-//               and the tcgen05.mma instructions, committing each stage to its "empty" barrier.
+//   warp 1      owns TMEM; in the MMA-issuing CTA one lane waits on the stage barriers and
+//               issues tcgen05.cp of each scale chunk into a rotating TMEM slot and the
+//               tcgen05.mma instructions, committing each stage to its "empty" barrier.
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, round to bf16, stage 32 x 32
 //               blocks in a swizzled shared-memory buffer (two per warp) and TMA-store them to
 //               D.  With two accumulators in TMEM the next tile's MMAs overlap the epilogue;
@@ -87,7 +86,6 @@ struct GemmArgs {
     int* tail_claim;
     const int32_t* masked_m;  // masked layout: valid rows per expert [G]
     int max_m;                // masked layout: rows per expert slab
-    int prefetch;             // K steps the L2 prefetch of A and B runs ahead of the loads (0: off)
 };
 
 template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false,
@@ -138,38 +136,28 @@ struct GemmCfg {
     static constexpr int SFB_CHUNK = SCALED ? SFB_ATOMS * UT_WORDS * 512 : 0;
     static constexpr int SF_STAGE_BYTES = SFA_CHUNK + SFB_CHUNK;
 
-    // Tensor memory: ACC_BUFS fp32 accumulators of BN columns, then the scale slots.  Scales
-    // reach tensor memory in batches of SF_BATCH groups (one burst of copies per batch, so the
-    // tensor pipe switches between copies and MMAs once per batch instead of once per group),
-    // into two sets of SF_BATCH slots used alternately: batch b is copied while the MMAs of
-    // batch b - 1 may still read the other set.
+    // Tensor memory: ACC_BUFS fp32 accumulators of BN columns, then rotating scale slots.
+    // (Measured: loading the chunks of several groups at once into a separate two-slot ring and
+    // copying them in one burst was slower for FP8 and FP4 than this: the ring limited how far
+    // the loads could run ahead, and long bursts of copies stalled the MMAs.)
     static constexpr int TMEM_COLS = 512;
     static constexpr int ACC_COLS = ACC_BUFS * BN;
     static constexpr int SFA_COLS = UT_WORDS * 4;
     static constexpr int SFB_COLS = UT_WORDS * SFB_ATOMS * 4;
     static constexpr int SF_SLOT_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int SF_BATCH = !SCALED                                         ? 1
-                                    : ACC_COLS + 8 * SF_SLOT_COLS <= TMEM_COLS ? 4
-                                    : ACC_COLS + 4 * SF_SLOT_COLS <= TMEM_COLS ? 2
-                                                                               : 1;
-    static constexpr int SF_SLOTS = 2 * SF_BATCH;
-    static_assert(!SCALED || ACC_COLS + SF_SLOTS * SF_SLOT_COLS <= TMEM_COLS,
-                  "tensor memory too small for the scale slots");
-    static constexpr int SF_BATCH_KSTEPS = SF_BATCH * SF_PERIOD;  // K steps per batch
-    static constexpr int SF_BATCH_BYTES = SF_BATCH * SF_STAGE_BYTES;
+    static constexpr int SF_SLOTS_FIT = SCALED ? (TMEM_COLS - ACC_COLS) / SF_SLOT_COLS : 1;
+    static constexpr int SF_SLOTS = SF_SLOTS_FIT > 4 ? 4 : SF_SLOTS_FIT;
+    static_assert(!SCALED || SF_SLOTS >= 1, "tensor memory too small for the scale slots");
 
     // Shared memory map (offsets from a 1024-byte aligned base).
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    // scale ring: two batches of chunks (A chunks of the batch's groups, then B chunks), each
-    // loaded with the first A/B stage of its batch and released by its own barrier
-    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SF = OFF_B + STAGES * B_BYTES;  // a scale chunk buffer per stage
     // epilogue staging: per epilogue warp two 32 x 32 bf16 blocks (64-byte swizzle)
     static constexpr int EPI_BLOCK = 32 * 32 * 2;
-    static constexpr int OFF_EPI = ((OFF_SF + (SCALED ? 2 * SF_BATCH_BYTES : 0) + 1023) / 1024) * 1024;
-    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail
-    // gather [4]; scale ring empty [2]
-    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4 + 2;
+    static constexpr int OFF_EPI = ((OFF_SF + STAGES * SF_STAGE_BYTES + 1023) / 1024) * 1024;
+    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail gather
+    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // masked layout: valid m-blocks before each expert [G + 1] and the clamped counts [G]
@@ -363,7 +351,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* tmem_empty = tmem_full + 2;
     uint64_t* drain = tmem_empty + 2;
     uint64_t* gather = drain + 1;  // [4]: one per epilogue warp
-    uint64_t* sf_empty = gather + 4;  // [2]: scale ring slots
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -386,7 +373,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mbar_init(drain, 1);
         for (int w = 0; w < 4; ++w) mbar_init(&gather[w], 1);
-        for (int b = 0; b < 2; ++b) mbar_init(&sf_empty[b], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -460,7 +446,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t it = 0, bc = 0;  // K steps and scale batches issued
+            uint32_t it = 0;
             bool ok = true;
             bool prior_done = false;  // the scale chunks come from the kernel launched before
             // this CTA's rows of work item w: its K range, first A row, tile column and expert
@@ -496,35 +482,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 return t;
             };
-            // L2 prefetch: a cursor runs args.prefetch K steps ahead of the loads, across work
-            // items, and brings the A and B boxes of its K step into L2 (no shared memory), so
-            // that a load finds its tile in L2 instead of waiting for DRAM
-            int pw = worker, pkb = 0;
-            Item pt{};
-            bool pvalid = args.prefetch > 0 && worker < num_work;
-            if (pvalid) {
-                pt = item_of(pw, false);
-                pkb = pt.wk.kb0;
-            }
-            const auto prefetch_next = [&] {
-                if (!pvalid) return;
-                const int px = pkb * (C::kind == Kind::BF16 ? 64 : 128);
-                const int pnb0 = pt.n_blk * C::BN + (int)rank * C::BN_CTA;
-                tma_prefetch_2d(&tm_a, px, pt.m0);
-                if constexpr (C::GROUPED)
-                    tma_prefetch_3d(&tm_b, px, pnb0, pt.g);
-                else
-                    tma_prefetch_2d(&tm_b, px, pnb0);
-                if (++pkb >= pt.wk.kb1) {
-                    pw += workers;
-                    pvalid = pw < num_work;
-                    if (pvalid) {
-                        pt = item_of(pw, false);
-                        pkb = pt.wk.kb0;
-                    }
-                }
-            };
-            for (int i = 0; i < args.prefetch; ++i) prefetch_next();
             for (int w = worker; w < num_work && ok; w += workers) {
                 const Item cur = item_of(w, true);
                 const Work wk = cur.wk;
@@ -538,19 +495,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    // the first K step of every batch of scale groups also brings the batch's chunks
-                    const bool sf_here = C::SCALED && (kb - wk.kb0) % C::SF_BATCH_KSTEPS == 0;
-                    if (sf_here && !bounded_wait(&sf_empty[bc & 1u], ((bc >> 1) & 1u) ^ 1u, args, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    const bool sf_here = C::SCALED && kb % C::SF_PERIOD == 0;
                     if (leader)
                         mbar_arrive_expect_tx(&full[s], C::CTAS * (C::A_BYTES + C::B_BYTES +
-                                                                   (sf_here ? C::SF_BATCH_BYTES : 0)));
+                                                                   (sf_here ? C::SF_STAGE_BYTES : 0)));
                     uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
                     uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
-                    uint8_t* sf = smem + C::OFF_SF + (bc & 1u) * C::SF_BATCH_BYTES;
-                    if (sf_here) ++bc;
+                    uint8_t* sf = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
                     const int q = kb / C::SF_PERIOD;
@@ -566,12 +517,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         else
                             tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
                         if (sf_here) {
-                            // scale chunks of the batch's groups: this CTA's A rows, all BN B rows of the tile
+                            // scale chunks: this CTA's A rows, all BN B rows of the tile
                             tma_load_3d_pair(sf, &tm_sfa, lead_full, 0, m0 / C::BM, q);
                             if constexpr (C::GROUPED)
-                                tma_load_4d_pair(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q, g);
+                                tma_load_4d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q, g);
                             else
-                                tma_load_3d_pair(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q);
+                                tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, n_blk, q);
                         }
                     } else {
                         tma_load_2d(sa, &tm_a, &full[s], kx, m0);
@@ -582,12 +533,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         if (sf_here) {
                             tma_load_3d(sf, &tm_sfa, &full[s], 0, m0 / C::BM, q);
                             if constexpr (C::GROUPED)
-                                tma_load_4d(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q, g);
+                                tma_load_4d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q, g);
                             else
-                                tma_load_3d(sf + C::SF_BATCH * C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q);
+                                tma_load_3d(sf + C::SFA_CHUNK, &tm_sfb, &full[s], 0, n_blk, q);
                         }
                     }
-                    prefetch_next();
                 }
             }
             // Wind down: wait (bounded) until the copies issued for the last stages landed.
@@ -601,7 +551,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == 1 && leader) {
         // ------------------------------------------------------------ MMA issue (one lane)
         if (lane == 0) {
-            uint32_t it = 0, lt = 0, bc = 0;  // K steps, work items and scale batches issued
+            uint32_t it = 0, lt = 0, git = 0;  // K steps, work items and scale groups issued
             bool ok = true;
             for (int w = worker; w < num_work && ok; w += workers, ++lt) {
                 const Work wk =
@@ -614,7 +564,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * C::BN;
-                uint32_t slot = 0, slot_base = 0;
+                uint32_t slot = 0;
                 for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
@@ -624,47 +574,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     tc_fence_after();
                     if constexpr (C::SCALED) {
-                        const int rel = kb - wk.kb0;
-                        if (rel % C::SF_BATCH_KSTEPS == 0) {
-                            // copy the chunks of this batch's groups (carried in with this stage) into
-                            // the slot set bc % 2, one slot per group; copies and MMAs run in issue
-                            // order on the tensor pipe, so the MMAs that read the set two batches ago
-                            // were done before these copies overwrite it
-                            slot_base = (bc & 1u) * C::SF_BATCH;
-                            const uint8_t* sf = smem + C::OFF_SF + (bc & 1u) * C::SF_BATCH_BYTES;
+                        if (kb % C::SF_PERIOD == 0) {
+                            // copy this group's scale chunks (carried by this stage) into TMEM slot
+                            // git % SF_SLOTS; copies and MMAs run in issue order on the tensor pipe
+                            slot = git % C::SF_SLOTS;
+                            ++git;
+                            const uint32_t sfa_col = C::ACC_COLS + slot * C::SF_SLOT_COLS;
+                            const uint32_t sfb_col = sfa_col + C::SFA_COLS;
+                            const uint8_t* ua = smem + C::OFF_SF + s * C::SF_STAGE_BYTES;
+                            const uint8_t* ub = ua + C::SFA_CHUNK;
 #pragma unroll
-                            for (int i = 0; i < C::SF_BATCH; ++i) {
-                                if (kb + i * C::SF_PERIOD >= wk.kb1) break;
-                                const uint32_t sfa_col = C::ACC_COLS + (slot_base + i) * C::SF_SLOT_COLS;
-                                const uint32_t sfb_col = sfa_col + C::SFA_COLS;
-                                const uint8_t* ua = sf + i * C::SFA_CHUNK;
-                                const uint8_t* ub = sf + C::SF_BATCH * C::SFA_CHUNK + i * C::SFB_CHUNK;
+                            for (int u = 0; u < C::UT_WORDS; ++u) {
+                                if constexpr (C::PAIR)
+                                    tc_cp_32x128b_warpx4_pair(tmem_base + sfa_col + 4 * u,
+                                                              smem_desc_rows16(ua + u * 512));
+                                else
+                                    tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(ua + u * 512));
 #pragma unroll
-                                for (int u = 0; u < C::UT_WORDS; ++u) {
+                                for (int at = 0; at < C::SFB_ATOMS; ++at) {
+                                    const uint32_t col = tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at);
+                                    const uint64_t d = smem_desc_rows16(ub + (at * C::UT_WORDS + u) * 512);
                                     if constexpr (C::PAIR)
-                                        tc_cp_32x128b_warpx4_pair(tmem_base + sfa_col + 4 * u,
-                                                                  smem_desc_rows16(ua + u * 512));
+                                        tc_cp_32x128b_warpx4_pair(col, d);
                                     else
-                                        tc_cp_32x128b_warpx4(tmem_base + sfa_col + 4 * u, smem_desc_rows16(ua + u * 512));
-#pragma unroll
-                                    for (int at = 0; at < C::SFB_ATOMS; ++at) {
-                                        const uint32_t col = tmem_base + sfb_col + 4 * (u * C::SFB_ATOMS + at);
-                                        const uint64_t d = smem_desc_rows16(ub + (at * C::UT_WORDS + u) * 512);
-                                        if constexpr (C::PAIR)
-                                            tc_cp_32x128b_warpx4_pair(col, d);
-                                        else
-                                            tc_cp_32x128b_warpx4(col, d);
-                                    }
+                                        tc_cp_32x128b_warpx4(col, d);
                                 }
                             }
-                            // the ring slot is free once these copies (and the MMAs before them) are done
-                            if constexpr (C::PAIR)
-                                tc_commit_pair_mc(&sf_empty[bc & 1u], kPairMask);
-                            else
-                                tc_commit(&sf_empty[bc & 1u]);
-                            ++bc;
                         }
-                        slot = slot_base + (uint32_t)((rel % C::SF_BATCH_KSTEPS) / C::SF_PERIOD);
                     }
                     const uint64_t adesc = smem_desc_k_sw128(smem + C::OFF_A + s * C::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + s * C::B_BYTES);
@@ -896,106 +832,119 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                      (int64_t)((int)rank * C::BM + (int)quarter * 32) * C::BN;
                 const int P = 32 / S;  // rows per gather pass: P rows of all S slots fill the staging area
                 bool ok = true;
-                const int n_claims = (state & 1) ? ((state & 2) ? S : 1) : 0;
-                for (int i = 0; i < n_claims && ok; ++i) {
-                    const int share = (wk.slice + i) % S;
+                // shares this warp reduces (bit j: share j): its own first, claimed by lane 0; then,
+                // in the slice that published last, every share still open, claimed in one round
+                // (lane j tries share j) after its own is done, so the owners come first
+                uint32_t todo = 0;
+                if (state & 1) {
                     int won = 0;
-                    if (lane == 0) won = atomicCAS(claim + share, 0, 1) == 0;
-                    if (!__shfl_sync(0xffffffffu, won, 0)) continue;
-                    const int r_end = (share + 1) * 32 / S;
-                    for (int rp = share * 32 / S; rp < r_end; rp += P) {
-                        const int nr = r_end - rp < P ? r_end - rp : P;
-                        // the staging area's previous contents have been read by every lane
-                        __syncwarp();
-                        fence_proxy_async_smem();
-                        if (lane == 0) {
-                            mbar_arrive_expect_tx(&gather[warp - 2], (uint32_t)(nr * S * row_bytes));
-                            for (int r = 0; r < nr; ++r)
-                                for (int j = 0; j < S; ++j)
-                                    bulk_load(stage + (r * S + j) * row_bytes, wbase + j * slot_stride + (int64_t)(rp + r) * C::BN,
-                                              (uint32_t)row_bytes, &gather[warp - 2]);
-                        }
-                        if (!warp_wait(&gather[warp - 2], gather_phase, args, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        gather_phase ^= 1u;
-                        // The reduction runs once, at the end of the kernel, so its instructions are
-                        // cold: compact loops, not unrolled bodies.  First every row's S copies are
-                        // added, in slot order, into its slot-0 copy (16 bytes per lane, consecutive
-                        // lanes on consecutive bytes); then the sums are rounded and written.
-                        const uint32_t sbase = smem_u32(stage);
-                        const uint32_t row_pitch = (uint32_t)(S * row_bytes);  // between gathered rows
-#pragma unroll 1
-                        for (int r = 0; r < nr; ++r) {
-#pragma unroll 1
-                            for (int c = (int)lane * 4; c < C::BN; c += 128) {
-                                const uint32_t a0 = sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u;
-                                float4 acc = ld_shared_f32x4(a0);
-#pragma unroll 1
-                                for (int j = 1; j < S; ++j) {
-                                    const float4 x = ld_shared_f32x4(a0 + (uint32_t)(j * row_bytes));
-                                    acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
-                                }
-                                st_shared_f32x4(a0, acc);
+                    if (lane == 0) won = atomicCAS(claim + wk.slice, 0, 1) == 0;
+                    if (__shfl_sync(0xffffffffu, won, 0)) todo = 1u << wk.slice;
+                }
+                for (int round = 0; round < 2 && ok; ++round) {
+                    if (round == 1) {
+                        if (!(state & 2)) break;
+                        const bool took = (int)lane < S && (int)lane != wk.slice && atomicCAS(claim + lane, 0, 1) == 0;
+                        todo = __ballot_sync(0xffffffffu, took);
+                    }
+                    while (todo && ok) {
+                        const int share = __ffs(todo) - 1;
+                        todo &= todo - 1;
+                        const int r_end = (share + 1) * 32 / S;
+                        for (int rp = share * 32 / S; rp < r_end; rp += P) {
+                            const int nr = r_end - rp < P ? r_end - rp : P;
+                            // the staging area's previous contents have been read by every lane
+                            __syncwarp();
+                            fence_proxy_async_smem();
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(&gather[warp - 2], (uint32_t)(nr * S * row_bytes));
+                                for (int r = 0; r < nr; ++r)
+                                    for (int j = 0; j < S; ++j)
+                                        bulk_load(stage + (r * S + j) * row_bytes, wbase + j * slot_stride + (int64_t)(rp + r) * C::BN,
+                                                  (uint32_t)row_bytes, &gather[warp - 2]);
                             }
-                        }
-                        __syncwarp();
-                        if constexpr (C::TRANS_D) {
-                            // element (row, n0 + c) goes to D[n0 + c][row]: lane l writes D rows n0 + l,
-                            // n0 + l + 32, ..., each with the nr consecutive bf16 of its column, eight at
-                            // a time (one 16-byte store where D's row allows it)
-                            const int row0 = m0 + (int)quarter * 32 + rp;
-#pragma unroll 1
-                            for (int c = (int)lane; c < C::BN; c += 32) {
-                                const int d_row = n0 + c;
-                                if (d_row >= args.N) continue;
-                                __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
-#pragma unroll 1
-                                for (int r8 = 0; r8 < nr; r8 += 8) {
-                                    uint32_t w[4];
-#pragma unroll
-                                    for (int h = 0; h < 4; ++h) {
-                                        const int r = r8 + 2 * h;
-                                        const float lo = r < nr ? ld_shared_f32(sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u) : 0.f;
-                                        const float hi = r + 1 < nr ? ld_shared_f32(sbase + (uint32_t)(r + 1) * row_pitch + (uint32_t)c * 4u) : 0.f;
-                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(lo, hi));
-                                        w[h] = *reinterpret_cast<uint32_t*>(&b2);
-                                    }
-                                    __nv_bfloat16* d8 = dst + r8;
-                                    if (r8 + 8 <= nr && row0 + r8 + 8 <= args.M && (reinterpret_cast<uintptr_t>(d8) & 15u) == 0) {
-                                        *reinterpret_cast<uint4*>(d8) = make_uint4(w[0], w[1], w[2], w[3]);
-                                    } else {
-#pragma unroll
-                                        for (int r = 0; r < 8; ++r)
-                                            if (r8 + r < nr && row0 + r8 + r < args.M)
-                                                *reinterpret_cast<uint16_t*>(d8 + r) = (uint16_t)(w[r >> 1] >> (16 * (r & 1)));
-                                    }
-                                }
+                            if (!warp_wait(&gather[warp - 2], gather_phase, args, abort_flag)) {
+                                ok = false;
+                                break;
                             }
-                        } else {
-                            const int col = (int)lane * 8;  // 8 columns per lane
-                            const int n = n0 + col;
+                            gather_phase ^= 1u;
+                            // The reduction runs once, at the end of the kernel, so its instructions are
+                            // cold: compact loops, not unrolled bodies.  First every row's S copies are
+                            // added, in slot order, into its slot-0 copy (16 bytes per lane, consecutive
+                            // lanes on consecutive bytes); then the sums are rounded and written.
+                            const uint32_t sbase = smem_u32(stage);
+                            const uint32_t row_pitch = (uint32_t)(S * row_bytes);  // between gathered rows
 #pragma unroll 1
                             for (int r = 0; r < nr; ++r) {
-                                const int row = m0 + (int)quarter * 32 + rp + r;
-                                if (row >= args.M || col >= C::BN || n >= args.N) continue;
-                                const uint32_t a4 = sbase + (uint32_t)r * row_pitch + (uint32_t)col * 4u;
-                                const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
-                                const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                                __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
-                                if (n + 8 <= args.N) {
-                                    uint32_t o[4];
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(v[2 * e], v[2 * e + 1]));
-                                        o[e] = *reinterpret_cast<uint32_t*>(&b2);
+#pragma unroll 1
+                                for (int c = (int)lane * 4; c < C::BN; c += 128) {
+                                    const uint32_t a0 = sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u;
+                                    float4 acc = ld_shared_f32x4(a0);
+#pragma unroll 1
+                                    for (int j = 1; j < S; ++j) {
+                                        const float4 x = ld_shared_f32x4(a0 + (uint32_t)(j * row_bytes));
+                                        acc.x += x.x, acc.y += x.y, acc.z += x.z, acc.w += x.w;
                                     }
-                                    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-                                } else {
+                                    st_shared_f32x4(a0, acc);
+                                }
+                            }
+                            __syncwarp();
+                            if constexpr (C::TRANS_D) {
+                                // element (row, n0 + c) goes to D[n0 + c][row]: lane l writes D rows n0 + l,
+                                // n0 + l + 32, ..., each with the nr consecutive bf16 of its column, eight at
+                                // a time (one 16-byte store where D's row allows it)
+                                const int row0 = m0 + (int)quarter * 32 + rp;
+#pragma unroll 1
+                                for (int c = (int)lane; c < C::BN; c += 32) {
+                                    const int d_row = n0 + c;
+                                    if (d_row >= args.N) continue;
+                                    __nv_bfloat16* dst = args.D + (int64_t)d_row * args.ldd + row0;
+#pragma unroll 1
+                                    for (int r8 = 0; r8 < nr; r8 += 8) {
+                                        uint32_t w[4];
 #pragma unroll
-                                    for (int e = 0; e < 8; ++e)
-                                        if (n + e < args.N) dst[e] = __float2bfloat16_rn(v[e]);
+                                        for (int h = 0; h < 4; ++h) {
+                                            const int r = r8 + 2 * h;
+                                            const float lo = r < nr ? ld_shared_f32(sbase + (uint32_t)r * row_pitch + (uint32_t)c * 4u) : 0.f;
+                                            const float hi = r + 1 < nr ? ld_shared_f32(sbase + (uint32_t)(r + 1) * row_pitch + (uint32_t)c * 4u) : 0.f;
+                                            __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(lo, hi));
+                                            w[h] = *reinterpret_cast<uint32_t*>(&b2);
+                                        }
+                                        __nv_bfloat16* d8 = dst + r8;
+                                        if (r8 + 8 <= nr && row0 + r8 + 8 <= args.M && (reinterpret_cast<uintptr_t>(d8) & 15u) == 0) {
+                                            *reinterpret_cast<uint4*>(d8) = make_uint4(w[0], w[1], w[2], w[3]);
+                                        } else {
+#pragma unroll
+                                            for (int r = 0; r < 8; ++r)
+                                                if (r8 + r < nr && row0 + r8 + r < args.M)
+                                                    *reinterpret_cast<uint16_t*>(d8 + r) = (uint16_t)(w[r >> 1] >> (16 * (r & 1)));
+                                        }
+                                    }
+                                }
+                            } else {
+                                const int col = (int)lane * 8;  // 8 columns per lane
+                                const int n = n0 + col;
+#pragma unroll 1
+                                for (int r = 0; r < nr; ++r) {
+                                    const int row = m0 + (int)quarter * 32 + rp + r;
+                                    if (row >= args.M || col >= C::BN || n >= args.N) continue;
+                                    const uint32_t a4 = sbase + (uint32_t)r * row_pitch + (uint32_t)col * 4u;
+                                    const float4 x0 = ld_shared_f32x4(a4), x1 = ld_shared_f32x4(a4 + 16);
+                                    const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                                    __nv_bfloat16* dst = args.D + (int64_t)row * args.ldd + n;
+                                    if (n + 8 <= args.N) {
+                                        uint32_t o[4];
+#pragma unroll
+                                        for (int e = 0; e < 4; ++e) {
+                                            __nv_bfloat162 b2 = __float22bfloat162_rn(make_float2(v[2 * e], v[2 * e + 1]));
+                                            o[e] = *reinterpret_cast<uint32_t*>(&b2);
+                                        }
+                                        *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+                                    } else {
+#pragma unroll
+                                        for (int e = 0; e < 8; ++e)
+                                            if (n + e < args.N) dst[e] = __float2bfloat16_rn(v[e]);
+                                    }
                                 }
                             }
                         }

@@ -34,9 +34,6 @@
  *     device, and free it on the same stream.  Every call can be captured in a CUDA graph;
  *     under capture the scratch becomes a graph memory node.
  *   - Results are deterministic: the same inputs give the same bytes on every run.
- *   - The GEMMs bring their operand tiles into L2 a few K steps ahead of loading them; the
- *     environment variable BSP_L2_PREFETCH_KSTEPS (read once per process, 0..64, 0 = off)
- *     sets how many.  It changes timing only, never results.
  *
  * Packed scale-factor layout ("SF words"): for a matrix with MN scale rows and KB scale
  * blocks along K, the SF tensor is int16 [ceil(KB/2)][ld], with
