@@ -121,17 +121,17 @@ int max_workers_of(const DeviceCtx& ctx, int* out) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = C::CTAS;
+        attr[0].val.clusterDim.x = C::CLUSTER;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.blockDim = dim3(C::THREADS);
         cfg.dynamicSmemBytes = C::SMEM_BYTES;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cfg.gridDim = dim3(C::CTAS * (ctx.sms / C::CTAS));
+        cfg.gridDim = dim3(C::CLUSTER * (ctx.sms / C::CLUSTER));
         int clusters = 0;
         if (err[dev] == cudaSuccess) err[dev] = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<C>, &cfg);
-        workers[dev] = clusters > 0 ? clusters : ctx.sms / C::CTAS;
+        workers[dev] = clusters > 0 ? clusters : ctx.sms / C::CLUSTER;
     });
     if (err[dev] != cudaSuccess) return BSP_ERR_CUDA;
     *out = workers[dev];
@@ -215,7 +215,7 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C::CTAS;
+    attr[0].val.clusterDim.x = C::CLUSTER;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     // Scaled kinds follow their own scale layout pass on the stream: the GEMM may launch while
@@ -227,7 +227,7 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = C::SCALED ? 2 : 1;
-    cfg.gridDim = dim3(C::CTAS * workers);
+    cfg.gridDim = dim3(C::CLUSTER * workers);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<C>, ta, tb, tsa, tsb, td, tw, a);
     g_launches.fetch_add(1);
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? BSP_OK : BSP_ERR_CUDA;
@@ -259,6 +259,10 @@ using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 using CfgBF16S = GemmCfg<Kind::BF16, 128, 8, false, true, 2, false, true>;
 using CfgFP8S = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true>;
 using CfgFP4S = GemmCfg<Kind::FP4, 128, 7, false, true, 2, false, true>;
+// M <= 128 whose transposed tiles would all be cut into two K slices: the two halves of a tile
+// run on the two CTA pairs of a 4-CTA cluster and meet in distributed shared memory instead of
+// a global workspace (one tile per cluster)
+using CfgFP8S2 = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true, true>;
 
 // Tile shape by problem shape.  M > 128: CTA pairs, 256 or 224 columns wide, whichever
 // finishes first by a model of the waves (tile time proportional to its MMA work, 224-wide
@@ -394,7 +398,7 @@ int plan_gemm(GemmArgs& a, const DeviceCtx& ctx, TailPlan* p, int* workers) {
     a.n_blocks = (a.N + C::BN - 1) / C::BN;
     int max_workers = 0;
     BSP_TRY(max_workers_of<C>(ctx, &max_workers));
-    *p = plan_tail(a.m_blocks * a.n_blocks, a.num_kb, C::SF_PERIOD, max_workers, !C::GROUPED);
+    *p = plan_tail(a.m_blocks * a.n_blocks, a.num_kb, C::SF_PERIOD, max_workers, !C::GROUPED && !C::CSPLIT);
     if constexpr (C::PAIR_LIST) {
         // the pair tiles are found on the device: between M/256 and M/128 of them per column block;
         // the grid is sized for the most
@@ -402,6 +406,19 @@ int plan_gemm(GemmArgs& a, const DeviceCtx& ctx, TailPlan* p, int* workers) {
     }
     *workers = max_workers;
     return BSP_OK;
+}
+
+// True when config C would cut every tile of this (transposed) problem into exactly two K
+// slices and the tiles fit as co-resident clusters of the cluster-split config C2.
+template <class C, class C2>
+bool use_cluster_split(const GemmArgs& a, const DeviceCtx& ctx) {
+    GemmArgs t = a;
+    TailPlan p;
+    int max_workers = 0, clusters = 0;
+    if (plan_gemm<C>(t, ctx, &p, &max_workers) != BSP_OK) return false;
+    if (p.splits != 2 || p.full_tiles != 0) return false;
+    if (max_workers_of<C2>(ctx, &clusters) != BSP_OK) return false;
+    return p.tiles <= clusters;
 }
 
 template <class C>
@@ -418,6 +435,7 @@ int describe_plan(int M, int N, int K, const DeviceCtx& ctx, int32_t* out) {
     out[4] = p.num_work;
     out[5] = p.num_work < max_workers ? p.num_work : max_workers;
     out[6] = 0;
+    out[7] = 0;
     return BSP_OK;
 }
 
@@ -563,6 +581,8 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
         default: {  // Swap: M <= 128
             Operands os = o;
             swap_operands(os, a);
+            if (use_cluster_split<CfgFP8S, CfgFP8S2>(a, ctx))
+                return launch_gemm<CfgFP8S2>(os, a, ctx, stream, scratch, scratch_bytes);
             return launch_gemm<CfgFP8S>(os, a, ctx, stream, scratch, scratch_bytes);
         }
     }
@@ -630,6 +650,7 @@ int gemm_fp8_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
         default: {  // Swap: M <= 128
             Operands os = o;
             swap_operands(os, a);
+            if (use_cluster_split<CfgFP8S, CfgFP8S2>(a, *ctx)) return launch_gemm<CfgFP8S2>(os, a, *ctx, st);
             return launch_gemm<CfgFP8S>(os, a, *ctx, st);
         }
     }
@@ -793,6 +814,9 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                 default: {  // Swap: M <= 128
                     BSP_TRY(describe_plan<CfgFP8S>(N, M, K, *ctx, plan));
                     plan[6] = 1;
+                    GemmArgs t{};
+                    t.M = N, t.N = M, t.K = K;
+                    plan[7] = use_cluster_split<CfgFP8S, CfgFP8S2>(t, *ctx) ? 1 : 0;
                     return BSP_OK;
                 }
             }

@@ -89,7 +89,7 @@ struct GemmArgs {
 };
 
 template <Kind KIND, int BLOCK_N_, int STAGES_, bool GROUPED_, bool PAIR_, int ACC_BUFS_ = 2, bool MASKED_ = false,
-          bool TRANS_D_ = false>
+          bool TRANS_D_ = false, bool CSPLIT_ = false>
 struct GemmCfg {
     static constexpr Kind kind = KIND;
     static constexpr bool PAIR = PAIR_;
@@ -115,6 +115,11 @@ struct GemmCfg {
     // long N dimension on the 256-row pair tiles
     static constexpr bool TRANS_D = TRANS_D_;
     static_assert(!TRANS_D || !GROUPED, "transposed output: dense configs only");
+    // a tile's two K halves on the two CTA pairs of one 4-CTA cluster: pair 1 hands its fp32 sums
+    // to pair 0 through distributed shared memory (one tile per cluster, transposed output)
+    static constexpr bool CSPLIT = CSPLIT_;
+    static_assert(!CSPLIT || (PAIR_ && TRANS_D_ && ACC_BUFS_ == 2 && BLOCK_N_ == 128), "cluster split");
+    static constexpr int CLUSTER = CSPLIT ? 4 : (PAIR_ ? 2 : 1);  // CTAs per cluster
     static constexpr bool SCALED = KIND != Kind::BF16;
     // TMEM accumulators: two let the next tile's MMAs run under this tile's epilogue; with one,
     // the epilogue reads the whole accumulator into registers first and releases it at once
@@ -194,6 +199,13 @@ __device__ __forceinline__ Work work_of(const GemmArgs& a, int w, int period) {
     const int groups = (a.num_kb + period - 1) / period;
     const int g0 = j * groups / a.splits, g1 = (j + 1) * groups / a.splits;
     return Work{a.full_tiles + tail, g0 * period, min(g1 * period, a.num_kb), tail, j};
+}
+
+// Cluster split: tile w, K half `half` (split at a scale-group boundary, as work_of cuts two slices).
+__device__ __forceinline__ Work half_work(const GemmArgs& a, int w, int half, int period) {
+    const int groups = (a.num_kb + period - 1) / period;
+    const int mid = min(groups / 2 * period, a.num_kb);
+    return half == 0 ? Work{w, 0, mid, -1, 0} : Work{w, mid, a.num_kb, -1, 1};
 }
 
 // Masked layout: work item w is n-block w % n_blocks of the (w / n_blocks)-th valid 128-row
@@ -356,11 +368,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const uint32_t lane = threadIdx.x % 32;
-    const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+    const uint32_t crank = C::PAIR ? cluster_ctarank() : 0u;  // rank in the cluster
+    const uint32_t rank = crank & 1u;                          // rank in the CTA pair
+    const uint32_t pairbase = crank & ~1u;                     // cluster rank of the pair's leader
     const bool leader = rank == 0;
-    const int worker = blockIdx.x / C::CTAS;
-    const int workers = gridDim.x / C::CTAS;
-    constexpr uint16_t kPairMask = 0x3;
+    const int worker = blockIdx.x / C::CLUSTER;
+    const int workers = gridDim.x / C::CLUSTER;
+    const uint16_t kPairMask = (uint16_t)(0x3u << pairbase);
+    const int half = C::CSPLIT ? (int)(crank >> 1) : 0;  // cluster split: this pair's K half
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -468,7 +483,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         t.g = 0;
                     }
                 } else {
-                    t.wk = work_of(args, w, C::SF_PERIOD);
+                    t.wk = C::CSPLIT ? half_work(args, w, half, C::SF_PERIOD) : work_of(args, w, C::SF_PERIOD);
                     const Tile tl = tile_of(args, t.wk.tile);
                     t.m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
                     t.n_blk = tl.n_blk;
@@ -510,7 +525,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         prior_done = true;
                     }
                     if constexpr (C::PAIR) {
-                        const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), 0);
+                        const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), pairbase);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
                         if constexpr (C::GROUPED)
                             tma_load_3d_pair(sb, &tm_b, lead_full, kx, nb0, g);
@@ -555,7 +570,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bool ok = true;
             for (int w = worker; w < num_work && ok; w += workers, ++lt) {
                 const Work wk =
-                    (C::MASKED || C::PAIR_LIST) ? Work{0, 0, args.num_kb, -1, 0} : work_of(args, w, C::SF_PERIOD);
+                    (C::MASKED || C::PAIR_LIST) ? Work{0, 0, args.num_kb, -1, 0}
+                    : C::CSPLIT                 ? half_work(args, w, half, C::SF_PERIOD)
+                                                : work_of(args, w, C::SF_PERIOD);
                 const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
                 const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
                 if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
@@ -661,7 +678,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t quarter = warp % 4;  // TMEM lanes this warp may read
         uint8_t* epi = smem + C::OFF_EPI + (warp - 2) * 2 * C::EPI_BLOCK;
         uint32_t lt = 0, nblk = 0, gather_phase = 0;
-        for (int w = worker; w < num_work; w += workers, ++lt) {
+        for (int w = C::CSPLIT ? num_work : worker; w < num_work; w += workers, ++lt) {
             Work wk{0, 0, args.num_kb, -1, 0};
             int m0, n_blk, g = 0;
             bool mine = true;  // this CTA's rows belong to the tile (false: the peer half of a one-block pair tile)
@@ -708,7 +725,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (leader)
                         mbar_arrive(&tmem_empty[buf]);
                     else
-                        mbar_arrive_remote(mapa_shared(smem_u32(&tmem_empty[buf]), 0));
+                        mbar_arrive_remote(mapa_shared(smem_u32(&tmem_empty[buf]), pairbase));
                 }
             };
             const auto pack = [&](uint32_t lo, uint32_t hi) -> uint32_t {
@@ -980,6 +997,80 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
+    }
+
+    if constexpr (C::CSPLIT) {
+        // One tile per cluster: pair h holds the fp32 sums of K half h in TMEM.  Every warp of the
+        // four CTAs passes the two cluster barriers below.  After the first, both pairs' MMAs are
+        // done (so the stage buffers are idle); pair 1's epilogue warps then store their sums into
+        // the stage buffers of the CTA of pair 0 with the same rank (128-byte swizzled 32 x 32
+        // blocks, the layout both sides index the same way); after the second, pair 0 adds them to
+        // its own, half 0 first, rounds to bf16 and writes D^T as the transposed epilogue does.
+        const bool epi = warp >= 2 && worker < num_work;
+        const uint32_t quarter = warp % 4;
+        bool ok = true;
+        int m0 = 0, n0 = 0;
+        if (epi) {
+            const Tile tl = tile_of(args, worker);
+            m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
+            n0 = tl.n_blk * C::BN;
+            ok = warp_wait(&tmem_full[0], 0, args, abort_flag);
+            tc_fence_after();
+        }
+        tc_fence_before();
+        cluster_sync();
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((quarter * 32) << 16);
+        uint8_t* xbuf = smem + C::OFF_A + (warp - 2) * (32 * C::BN * 4);  // 16 KB per epilogue warp
+        if (epi && ok && half == 1) {
+            const uint32_t dst = mapa_shared(smem_u32(xbuf), crank - 2u);
+#pragma unroll 1
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    st_shared_cluster_u32x4(dst + (uint32_t)(c * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)), r[4 * v],
+                                            r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            }
+        }
+        tc_fence_before();
+        cluster_sync();
+        tc_fence_after();
+        if (epi && ok && half == 0) {
+            const int row = m0 + (int)(quarter * 32 + lane);
+            const uint32_t xb = smem_u32(xbuf);
+#pragma unroll 1
+            for (int c = 0; c < C::BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(taddr + c * 32, r);
+                tmem_ld_wait();
+                uint32_t w16[16];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 x = ld_shared_f32x4(xb + (uint32_t)(c * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)));
+                    const float s0 = __uint_as_float(r[4 * v]) + x.x, s1 = __uint_as_float(r[4 * v + 1]) + x.y;
+                    const float s2 = __uint_as_float(r[4 * v + 2]) + x.z, s3 = __uint_as_float(r[4 * v + 3]) + x.w;
+                    __nv_bfloat162 b0 = __float22bfloat162_rn(make_float2(s0, s1));
+                    __nv_bfloat162 b1 = __float22bfloat162_rn(make_float2(s2, s3));
+                    w16[2 * v] = *reinterpret_cast<uint32_t*>(&b0);
+                    w16[2 * v + 1] = *reinterpret_cast<uint32_t*>(&b1);
+                }
+                // element (row, n0 + 32c + j) goes to D[n0 + 32c + j][row]: for each j the warp writes
+                // 32 consecutive bf16 of one row of D
+                if (row < args.M) {
+                    __nv_bfloat16* col = args.D + row;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int d_row = n0 + c * 32 + j;
+                        if (d_row < args.N)
+                            *reinterpret_cast<uint16_t*>(col + (int64_t)d_row * args.ldd) =
+                                (uint16_t)(w16[j >> 1] >> (16 * (j & 1)));
+                    }
+                }
+            }
+        }
     }
 
     tc_fence_before();

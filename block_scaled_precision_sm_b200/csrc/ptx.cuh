@@ -181,6 +181,12 @@ __device__ __forceinline__ void st_shared_f32x4(uint32_t addr, float4 v) {
                  : "memory");
 }
 
+// 16-byte store into the shared memory of a CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void st_shared_cluster_u32x4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");

@@ -265,7 +265,7 @@ _PLAN_KINDS = {"bf16": 0, "fp8": 1, "fp4": 2, "grouped_fp8": 3}
 
 def gemm_plan(kind: str, M: int, N: int, K: int) -> dict:
     """How the library would launch this GEMM on the current device (nothing is launched)."""
-    out = (ctypes.c_int32 * 7)()
+    out = (ctypes.c_int32 * 8)()
     _lib.call("bsp_gemm_plan", _PLAN_KINDS[kind], M, N, K, ctypes.cast(out, ctypes.c_void_p))
-    keys = ("tile_m", "tile_n", "splits", "split_tiles", "work_items", "workers", "transposed")
+    keys = ("tile_m", "tile_n", "splits", "split_tiles", "work_items", "workers", "transposed", "cluster_split")
     return dict(zip(keys, (int(v) for v in out)))

@@ -238,12 +238,15 @@ uint64_t bsp_set_wait_timeout_ns(uint64_t ns);
 /*
  * bsp_gemm_plan — how a GEMM of this kind and shape would be launched on the current
  * device, without launching it.  kind: 0 BF16, 1 FP8 (gemm_fp8_nt), 2 FP4, 3 M-grouped FP8
- * (M = M_total).  Writes seven int32 to `plan` (caller-owned host memory):
+ * (M = M_total).  Writes eight int32 to `plan` (caller-owned host memory):
  *   plan[0] rows per tile (128 single CTA, 256 CTA pair)   plan[1] columns per tile
  *   plan[2] K slices per split tile (1: no split)          plan[3] split tiles
  *   plan[4] work items (whole tiles + slices)              plan[5] persistent workers launched
- *   plan[6] 1 if the product is computed transposed, D^T = B A^T (FP8 with M <= 128: the
- *           tile rows then run along N and the columns along M), else 0
+ *   plan[6] 1 if the product is computed transposed, D^T = B A^T (M <= 128: the tile rows
+ *           then run along N and the columns along M), else 0
+ *   plan[7] 1 if the two K slices of every tile run on the two CTA pairs of one 4-CTA cluster
+ *           and are added in distributed shared memory (FP8, M <= 128, two slices per tile,
+ *           all tiles co-resident), else 0; the sums and their order are the same either way
  * The tiles left after the last full wave of workers are cut along K into slices at
  * scale-group boundaries when that shortens the last wave (at least two slices of eight or
  * more K steps); their fp32 partial sums meet in a workspace and are added in slice order

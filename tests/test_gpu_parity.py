@@ -230,6 +230,23 @@ def test_fp8_small_m_runs_transposed(ops, orc, m, n, k, gran):
     _fp8_case(ops, orc, m, n, k, seed=m * 13 + n, gran=gran)
 
 
+# M <= 128 whose transposed tiles are all cut into two K slices: the two halves run on the two
+# CTA pairs of a 4-CTA cluster and meet in distributed shared memory (ragged N along the tile rows,
+# M below 32 and not a multiple of 8, per-row and 128x128 B scales)
+@pytest.mark.parametrize("m,n,k,gran", [(128, 7168, 2048, 128), (100, 5000, 2048, 1), (17, 7000, 4096, 128),
+                                        (128, 1024, 2048, 1)])
+def test_fp8_small_m_cluster_split(ops, orc, m, n, k, gran):
+    plan = ops.gemm_plan("fp8", m, n, k)
+    assert plan["cluster_split"] == 1 and plan["splits"] == 2 and plan["transposed"] == 1, plan
+    _fp8_case(ops, orc, m, n, k, seed=m * 3 + n, gran=gran)
+    p = inputs.dense_fp8_problem(m, n, k, seed=5, b_block_rows=gran)
+    args = [to_dev(p[x]) for x in ("A", "sfa", "B", "sfb")]
+    d1 = ops.gemm_fp8_nt(*args, sfb_gran_n=gran)
+    d2 = ops.gemm_fp8_nt(*args, sfb_gran_n=gran)
+    _status_ok(ops)
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
 @pytest.mark.parametrize("kind,m,n,k", [("bf16", 128, 3000, 2048), ("bf16", 5, 448, 640), ("fp4", 128, 2000, 4096),
                                         ("fp4", 40, 704, 1024)])
 def test_bf16_fp4_small_m_run_transposed(ops, orc, kind, m, n, k):

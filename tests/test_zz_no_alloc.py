@@ -4,9 +4,9 @@ It is called here through the C ABI, as such a caller would, and its output is c
 against the fp64 oracle and against the regular gemm_fp8_nt path on the same inputs, on two
 calls in a row with different data (the second call reuses the shared scratch the first one
 left behind).  The shapes cover each way the call can run: CTA-pair tiles; the transposed
-small-M path with per-row B scales; a split last wave whose partial sums fit in the fixed
-scratch; and the full 4096 x 7168 x 16384 problem, whose split workspace would not fit, so the
-last wave runs unsplit.  This file is collected last so a stop-at-first-failure run has
+small-M path with per-row B scales, with its two K halves on one cluster, and with a split
+last wave whose partial sums fit in the fixed scratch; and the full 4096 x 7168 x 16384
+problem, whose split workspace would not fit, so the last wave runs unsplit.  This file is collected last so a stop-at-first-failure run has
 already run everything else.
 """
 
@@ -56,7 +56,8 @@ def _split_ws_bytes(plan):
 CASES = [
     (384, 672, 1024, 128, "pair, whole tiles"),
     (96, 1000, 1024, 1, "transposed, per-row B scales"),
-    (128, 1024, 2048, 1, "transposed, split tail in the fixed scratch"),
+    (128, 1024, 2048, 1, "transposed, K halves in a cluster"),
+    (33, 296, 4096, 1, "transposed, split tail in the fixed scratch"),
     (4096, 7168, 16384, 128, "pair, split workspace too large: unsplit"),
 ]
 
@@ -73,7 +74,9 @@ def test_noalloc_matches_oracle_and_regular_entry_point_twice(env, orc, m, n, k,
     if "whole" in path:
         assert plan["splits"] == 1, plan
     if "fixed scratch" in path:
-        assert plan["splits"] > 1 and _split_ws_bytes(plan) < SCRATCH_BYTES // 2, plan
+        assert plan["splits"] > 1 and not plan["cluster_split"] and _split_ws_bytes(plan) < SCRATCH_BYTES // 2, plan
+    if "cluster" in path:
+        assert plan["splits"] == 2 and plan["cluster_split"] == 1, plan
     if "too large" in path:
         assert plan["splits"] > 1 and _split_ws_bytes(plan) > SCRATCH_BYTES, plan
     p = inputs.dense_fp8_problem(m, n, k, seed=21, b_block_rows=gran)
