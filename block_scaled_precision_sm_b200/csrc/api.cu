@@ -182,9 +182,16 @@ int64_t tail_count_bytes(const TailPlan& p) {
 template <class C>
 int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
            GemmArgs a, const TailPlan& p, float* ws, int* count, const DeviceCtx& ctx, cudaStream_t stream) {
-    // D: bf16 [M][ldd], stored in 32 x 32 blocks through a 64-byte-swizzled staging buffer
+    // D: bf16 [M][ldd], stored in 32 x 32 blocks through a 64-byte-swizzled staging buffer; the
+    // cluster split of a transposed problem stores 64 rows x 32 columns of D (the swapped
+    // problem's N x M) from plain row-major blocks
     CUtensorMap td, tw;
-    {
+    if constexpr (C::CSPLIT) {
+        const cuuint64_t dims[2] = {(cuuint64_t)a.M, (cuuint64_t)a.N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(a.ldd * 2)};
+        const cuuint32_t box[2] = {32, (cuuint32_t)C::X_COLS};
+        BSP_TRY(encode(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.D, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    } else {
         const cuuint64_t dims[2] = {(cuuint64_t)a.N, (cuuint64_t)a.M};
         const cuuint64_t strides[1] = {(cuuint64_t)(a.ldd * 2)};
         const cuuint32_t box[2] = {32, 32};

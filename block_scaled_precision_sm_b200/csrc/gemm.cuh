@@ -161,8 +161,15 @@ struct GemmCfg {
     // epilogue staging: per epilogue warp two 32 x 32 bf16 blocks (64-byte swizzle)
     static constexpr int EPI_BLOCK = 32 * 32 * 2;
     static constexpr int OFF_EPI = ((OFF_SF + STAGES * SF_STAGE_BYTES + 1023) / 1024) * 1024;
-    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail gather
-    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
+    // full, empty [STAGES]; tmem_full, tmem_empty [2]; drain; per epilogue warp: split-tail
+    // gather; cluster split, per epilogue warp: receive buffer free, columns received
+    static constexpr int NUM_BARS = 2 * STAGES + 5 + 4 + (CSPLIT ? 8 : 0);
+    // cluster split, per epilogue warp: the 32 x 64 fp32 columns sent and those received, then
+    // its 64 x 32 bf16 block of D, in the idle A stage buffers
+    static constexpr int X_COLS = BN / 2;
+    static constexpr int X_BYTES = 32 * X_COLS * 4;
+    static constexpr int X_WARP_BYTES = 2 * X_BYTES + X_COLS * 32 * 2;
+    static_assert(!CSPLIT || 4 * X_WARP_BYTES <= STAGES * A_BYTES, "cluster-split buffers");
     static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BLOCK;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     // masked layout: valid m-blocks before each expert [G + 1] and the clamped counts [G]
@@ -363,6 +370,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* tmem_empty = tmem_full + 2;
     uint64_t* drain = tmem_empty + 2;
     uint64_t* gather = drain + 1;  // [4]: one per epilogue warp
+    uint64_t* xready = gather + 4;  // [4] (cluster split): the other pair's receive buffer is free
+    uint64_t* xfull = xready + 4;   // [4] (cluster split): the other pair's columns have arrived
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -388,6 +397,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mbar_init(drain, 1);
         for (int w = 0; w < 4; ++w) mbar_init(&gather[w], 1);
+        if constexpr (C::CSPLIT) {
+            for (int w = 0; w < 4; ++w) {
+                mbar_init(&xready[w], 1);
+                mbar_init(&xfull[w], 1);
+            }
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -1000,76 +1015,93 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
 
     if constexpr (C::CSPLIT) {
-        // One tile per cluster: pair h holds the fp32 sums of K half h in TMEM.  Every warp of the
-        // four CTAs passes the two cluster barriers below.  After the first, both pairs' MMAs are
-        // done (so the stage buffers are idle); pair 1's epilogue warps then store their sums into
-        // the stage buffers of the CTA of pair 0 with the same rank (128-byte swizzled 32 x 32
-        // blocks, the layout both sides index the same way); after the second, pair 0 adds them to
-        // its own, half 0 first, rounds to bf16 and writes D^T as the transposed epilogue does.
-        const bool epi = warp >= 2 && worker < num_work;
-        const uint32_t quarter = warp % 4;
-        bool ok = true;
-        int m0 = 0, n0 = 0;
-        if (epi) {
+        // One tile per cluster: pair h holds the fp32 sums of K half h in TMEM and finishes
+        // columns [64h, 64h + 64) of the tile.  Each epilogue warp trades 32 rows x 64 columns
+        // with the warp of the same quarter in the CTA of the other pair with the same rank:
+        // it announces that its receive buffer is free (its own MMAs are done, so the stage
+        // buffers are idle), lays out the columns the other pair finishes in its own shared
+        // memory and, once the other side's buffer is free, moves them there with one bulk copy
+        // that completes on the receiver's barrier.  It then adds the received sums to its own
+        // (the same fp32 sum of the two halves as the two-slice split tail), rounds to bf16 and
+        // stores its 64 x 32 block of D (rows of D are the tile's columns) with TMA.
+        if (warp >= 2 && worker < num_work) {
+            const uint32_t quarter = warp % 4;
+            const int wq = warp - 2;
             const Tile tl = tile_of(args, worker);
-            m0 = tl.m_blk * C::TILE_M + (int)rank * C::BM;
-            n0 = tl.n_blk * C::BN;
-            ok = warp_wait(&tmem_full[0], 0, args, abort_flag);
+            const int dcol = tl.m_blk * C::TILE_M + (int)rank * C::BM + (int)quarter * 32;  // columns of D
+            const int keep = half * C::X_COLS, give = (1 - half) * C::X_COLS;
+            const int drow = tl.n_blk * C::BN + keep;  // rows of D
+            uint8_t* sendb = smem + C::OFF_A + wq * C::X_WARP_BYTES;
+            uint8_t* recvb = sendb + C::X_BYTES;
+            uint8_t* outb = recvb + C::X_BYTES;
+            const uint32_t other = crank ^ 2u;
+            const uint32_t taddr = tmem_base + ((quarter * 32) << 16);
+            bool ok = warp_wait(&tmem_full[0], 0, args, abort_flag);
             tc_fence_after();
-        }
-        tc_fence_before();
-        cluster_sync();
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + ((quarter * 32) << 16);
-        uint8_t* xbuf = smem + C::OFF_A + (warp - 2) * (32 * C::BN * 4);  // 16 KB per epilogue warp
-        if (epi && ok && half == 1) {
-            const uint32_t dst = mapa_shared(smem_u32(xbuf), crank - 2u);
-#pragma unroll 1
-            for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int v = 0; v < 8; ++v)
-                    st_shared_cluster_u32x4(dst + (uint32_t)(c * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)), r[4 * v],
-                                            r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            if (ok && lane == 0) {
+                mbar_arrive_expect_tx(&xfull[wq], C::X_BYTES);
+                mbar_arrive_remote(mapa_shared(smem_u32(&xready[wq]), other));
             }
-        }
-        tc_fence_before();
-        cluster_sync();
-        tc_fence_after();
-        if (epi && ok && half == 0) {
-            const int row = m0 + (int)(quarter * 32 + lane);
-            const uint32_t xb = smem_u32(xbuf);
+            // lane l's 64 columns: 16 chunks of 16 bytes at l * 256, chunk v at v ^ (l & 15)
+            const auto chunk = [&](uint8_t* base, int v) {
+                return smem_u32(base) + lane * 256u + (uint32_t)((v ^ (int)(lane & 15)) << 4);
+            };
+            if (ok) {
 #pragma unroll 1
-            for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + c * 32, r);
-                tmem_ld_wait();
-                uint32_t w16[16];
+                for (int c = 0; c < C::X_COLS / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + give + c * 32, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 x = ld_shared_f32x4(xb + (uint32_t)(c * 4096 + lane * 128 + ((v ^ (lane & 7)) << 4)));
-                    const float s0 = __uint_as_float(r[4 * v]) + x.x, s1 = __uint_as_float(r[4 * v + 1]) + x.y;
-                    const float s2 = __uint_as_float(r[4 * v + 2]) + x.z, s3 = __uint_as_float(r[4 * v + 3]) + x.w;
-                    __nv_bfloat162 b0 = __float22bfloat162_rn(make_float2(s0, s1));
-                    __nv_bfloat162 b1 = __float22bfloat162_rn(make_float2(s2, s3));
-                    w16[2 * v] = *reinterpret_cast<uint32_t*>(&b0);
-                    w16[2 * v + 1] = *reinterpret_cast<uint32_t*>(&b1);
+                    for (int v = 0; v < 8; ++v)
+                        st_shared_f32x4(chunk(sendb, c * 8 + v),
+                                        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                 }
-                // element (row, n0 + 32c + j) goes to D[n0 + 32c + j][row]: for each j the warp writes
-                // 32 consecutive bf16 of one row of D
-                if (row < args.M) {
-                    __nv_bfloat16* col = args.D + row;
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (ok && lane == 0) {
+                ok = bounded_wait<true>(&xready[wq], 0, args, abort_flag);
+                if (ok)
+                    bulk_copy_to_cluster(mapa_shared(smem_u32(recvb), other), sendb, C::X_BYTES,
+                                         mapa_shared(smem_u32(&xfull[wq]), other));
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (ok) ok = warp_wait<true>(&xfull[wq], 0, args, abort_flag);
+            if (ok) {
+#pragma unroll 1
+                for (int c = 0; c < C::X_COLS / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + keep + c * 32, r);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int d_row = n0 + c * 32 + j;
-                        if (d_row < args.N)
-                            *reinterpret_cast<uint16_t*>(col + (int64_t)d_row * args.ldd) =
-                                (uint16_t)(w16[j >> 1] >> (16 * (j & 1)));
+                    for (int v = 0; v < 8; ++v) {
+                        const float4 x = ld_shared_f32x4(chunk(recvb, c * 8 + v));
+                        const float s0 = __uint_as_float(r[4 * v]) + x.x, s1 = __uint_as_float(r[4 * v + 1]) + x.y;
+                        const float s2 = __uint_as_float(r[4 * v + 2]) + x.z, s3 = __uint_as_float(r[4 * v + 3]) + x.w;
+                        __nv_bfloat162 b0 = __float22bfloat162_rn(make_float2(s0, s1));
+                        __nv_bfloat162 b1 = __float22bfloat162_rn(make_float2(s2, s3));
+                        const uint32_t w0 = *reinterpret_cast<uint32_t*>(&b0), w1 = *reinterpret_cast<uint32_t*>(&b1);
+                        // column 32c + 4v + i of the tile is row 32c + 4v + i of this block of D;
+                        // lane l is its column l (64 bytes a row)
+                        const uint32_t o = smem_u32(outb) + (uint32_t)((c * 32 + 4 * v) * 64) + lane * 2u;
+                        st_shared_u16(o, (uint16_t)w0);
+                        st_shared_u16(o + 64, (uint16_t)(w0 >> 16));
+                        st_shared_u16(o + 128, (uint16_t)w1);
+                        st_shared_u16(o + 192, (uint16_t)(w1 >> 16));
                     }
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                // rows past M and columns past N are dropped by the tensor map's bounds
+                if (lane == 0 && dcol < args.M && drow < args.N) {
+                    tma_store_2d(&tm_d, outb, dcol, drow);
+                    bulk_commit_group();
+                    bulk_wait_group_all();
+                }
             }
+            __syncwarp();
         }
     }
 

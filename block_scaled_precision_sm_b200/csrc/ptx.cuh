@@ -181,9 +181,18 @@ __device__ __forceinline__ void st_shared_f32x4(uint32_t addr, float4 v) {
                  : "memory");
 }
 
-// 16-byte store into the shared memory of a CTA of the cluster (shared::cluster address).
-__device__ __forceinline__ void st_shared_cluster_u32x4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from this CTA's shared
+// memory into the shared memory of a CTA of the cluster (`dst_cluster`, a shared::cluster
+// address); completion is counted in bytes on that CTA's barrier at `bar_cluster`.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                                     uint32_t bar_cluster) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
                  : "memory");
 }
 
