@@ -258,6 +258,7 @@ using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 // contiguous grouped layout on CTA pairs (pairs of 128-row blocks of one expert), used while the
 // block count fits the kernel's on-device tile list; CfgGrouped (single CTAs) otherwise
 using CfgGroupedPair = GemmCfg<Kind::FP8, 224, 6, true, true>;
+using CfgGroupedPair256 = GemmCfg<Kind::FP8, 256, 6, true, true, 1>;
 using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 // M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair, A's rows
 // across), written transposed.  Per SM and K step: 128 rows of B and 64 of A for 128 x 128
@@ -270,6 +271,13 @@ using CfgFP4S = GemmCfg<Kind::FP4, 128, 7, false, true, 2, false, true>;
 // run on the two CTA pairs of a 4-CTA cluster and meet in distributed shared memory instead of
 // a global workspace (one tile per cluster)
 using CfgFP8S2 = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true, true>;
+
+// Grouped pair tiles 256 columns wide unless 224-wide ones cover N with enough fewer wasted
+// columns to make up for being about 8% less efficient.
+bool grouped_wide(int N) {
+    const int64_t w256 = (int64_t)((N + 255) / 256) * 256, w224 = (int64_t)((N + 223) / 224) * 224;
+    return w256 * 23 <= w224 * 25;
+}
 
 // Tile shape by problem shape.  M > 128: CTA pairs, 256 or 224 columns wide, whichever
 // finishes first by a model of the waves (tile time proportional to its MMA work, 224-wide
@@ -716,8 +724,10 @@ int m_grouped_gemm_fp8_nt_contiguous(const void* A, const void* sfa, const void*
     a.D = static_cast<__nv_bfloat16*>(D), a.ldd = N;
     a.m_indices = m_indices, a.G = G;
     a.sfb_gran = sfb_gran_n;
-    if (M_total / 128 <= CfgGroupedPair::MAX_PAIR_TILES)
+    if (M_total / 128 <= CfgGroupedPair::MAX_PAIR_TILES) {
+        if (grouped_wide(N)) return launch_gemm<CfgGroupedPair256>(o, a, *ctx, static_cast<cudaStream_t>(stream));
         return launch_gemm<CfgGroupedPair>(o, a, *ctx, static_cast<cudaStream_t>(stream));
+    }
     return launch_gemm<CfgGrouped>(o, a, *ctx, static_cast<cudaStream_t>(stream));
 }
 
@@ -838,7 +848,9 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                 }
             }
         default:
-            if (M / 128 <= CfgGroupedPair::MAX_PAIR_TILES) return describe_plan<CfgGroupedPair>(M, N, K, *ctx, plan);
+            if (M / 128 <= CfgGroupedPair::MAX_PAIR_TILES)
+                return grouped_wide(N) ? describe_plan<CfgGroupedPair256>(M, N, K, *ctx, plan)
+                                       : describe_plan<CfgGroupedPair>(M, N, K, *ctx, plan);
             return describe_plan<CfgGrouped>(M, N, K, *ctx, plan);
     }
 }

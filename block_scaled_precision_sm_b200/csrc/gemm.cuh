@@ -535,10 +535,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     // x coordinate in elements of the tensor map's type: 64 bf16 or 128 bytes per step
                     const int kx = kb * (C::kind == Kind::BF16 ? 64 : 128);
                     const int q = kb / C::SF_PERIOD;
-                    if (sf_here && !prior_done) {
-                        griddep_wait();
-                        prior_done = true;
-                    }
+                    // A and B come from before the scale layout pass; its output is read only
+                    // once it has finished
+                    const auto await_prior = [&] {
+                        if (sf_here && !prior_done) {
+                            griddep_wait();
+                            prior_done = true;
+                        }
+                    };
                     if constexpr (C::PAIR) {
                         const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), pairbase);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
@@ -546,6 +550,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             tma_load_3d_pair(sb, &tm_b, lead_full, kx, nb0, g);
                         else
                             tma_load_2d_pair(sb, &tm_b, lead_full, kx, nb0);
+                        await_prior();
                         if (sf_here) {
                             // scale chunks: this CTA's A rows, all BN B rows of the tile
                             tma_load_3d_pair(sf, &tm_sfa, lead_full, 0, m0 / C::BM, q);
@@ -560,6 +565,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             tma_load_3d(sb, &tm_b, &full[s], kx, nb0, g);
                         else
                             tma_load_2d(sb, &tm_b, &full[s], kx, nb0);
+                        await_prior();
                         if (sf_here) {
                             tma_load_3d(sf, &tm_sfa, &full[s], 0, m0 / C::BM, q);
                             if constexpr (C::GROUPED)

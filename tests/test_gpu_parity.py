@@ -401,13 +401,16 @@ def test_grouped(ops, orc, counts, n, k):
     assert np.all(got[pad] == 0.0)  # padding rows are exactly zero
 
 
-def test_grouped_pair_tiles_odd_and_even_runs(ops, orc):
+# N = 448 runs on 224-wide pair tiles (two exactly); N = 512 and N = 1000 on 256-wide ones (the
+# latter with a ragged last tile), the accumulator then single-buffered
+@pytest.mark.parametrize("n,tile_n", [(448, 224), (512, 256), (1000, 256)])
+def test_grouped_pair_tiles_odd_and_even_runs(ops, orc, n, tile_n):
     # experts with 1, 2, 3, 1, 2, 0 and 5 blocks of 128 rows: pairs of blocks of one expert run on
     # CTA pairs, an odd last block alone (its peer CTA's rows, the next expert's, are not written)
     counts = [100, 256, 300, 1, 129, 0, 600]
-    p = inputs.grouped_fp8_problem(len(counts), sum(counts), 448, 512, seed=23, counts=counts)
-    plan = ops.gemm_plan("grouped_fp8", p["M"], 448, 512)
-    assert plan["tile_m"] == 256 and plan["tile_n"] == 224, plan
+    p = inputs.grouped_fp8_problem(len(counts), sum(counts), n, 512, seed=23, counts=counts)
+    plan = ops.gemm_plan("grouped_fp8", p["M"], n, 512)
+    assert plan["tile_m"] == 256 and plan["tile_n"] == tile_n, plan
     D = _grouped(ops, p)
     _status_ok(ops)
     got = bf16_to_f64(D)
