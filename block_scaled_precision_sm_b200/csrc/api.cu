@@ -260,6 +260,10 @@ using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 using CfgGroupedPair = GemmCfg<Kind::FP8, 224, 6, true, true>;
 using CfgGroupedPair256 = GemmCfg<Kind::FP8, 256, 6, true, true, 1>;
 using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
+// masked layout, transposed: 256 rows of an expert's B on a CTA pair against up to 256 of its
+// rows of A as the MMA's N (cut to the valid rows at run time), so B is streamed once per expert
+// (per 256 valid rows) instead of once per 128-row block
+using CfgMaskedT = GemmCfg<Kind::FP8, 256, 6, true, true, 1, true, true>;
 // M <= 128: computed as D^T = B A^T on 256 x 128 pair tiles (B's rows along the pair, A's rows
 // across), written transposed.  Per SM and K step: 128 rows of B and 64 of A for 128 x 128
 // products, against the same bytes for 128 x 64 in single-CTA narrow tiles: half the bytes per
@@ -334,6 +338,16 @@ struct ScaleChunks {
     int64_t a_bytes = 0, b_bytes = 0;
     ScaleChunks(const Operands& o, const GemmArgs& g) {
         const int q = (o.words + 2 * C::UT_WORDS - 1) / (2 * C::UT_WORDS);
+        if constexpr (C::MT) {
+            // A' = B_g (its scales per expert, 128-row tiles), B' = the rows of A (128-row atoms;
+            // a tile loads the two atoms of its chunk)
+            a = SfLayout{g.N, g.sfb_gran, o.words, o.ld_sfb, (int64_t)o.words * o.ld_sfb, C::BM, 1, C::UT_WORDS,
+                         (g.N + C::BM - 1) / C::BM, q, o.groups};
+            b = SfLayout{g.M, 1, o.words, o.ld_sfa, 0, 128, 1, C::UT_WORDS, (g.M + 127) / 128, q, 1};
+            a_bytes = round_up((int64_t)q * a.tiles * C::SFA_CHUNK * o.groups, 256);
+            b_bytes = round_up((int64_t)q * b.tiles * 512 * C::UT_WORDS, 256);
+            return;
+        }
         a = SfLayout{g.M, g.sfa_gran > 1 ? g.sfa_gran : 1, o.words, o.ld_sfa, 0, C::BM, 1, C::UT_WORDS,
                      (g.M + C::BM - 1) / C::BM, q, 1};
         const int64_t b_gstride = (int64_t)o.words * o.ld_sfb;
@@ -414,6 +428,11 @@ int plan_gemm(GemmArgs& a, const DeviceCtx& ctx, TailPlan* p, int* workers) {
     int max_workers = 0;
     BSP_TRY(max_workers_of<C>(ctx, &max_workers));
     *p = plan_tail(a.m_blocks * a.n_blocks, a.num_kb, C::SF_PERIOD, max_workers, !C::GROUPED && !C::CSPLIT);
+    if constexpr (C::MT) {
+        // masked transposed: at most ceil(max_m / 256) chunks per expert, found on the device
+        const int g = a.G > 0 ? a.G : 1, mm = a.G > 0 ? a.max_m : a.M;
+        p->tiles = p->full_tiles = p->num_work = g * ((mm + C::MCHUNK - 1) / C::MCHUNK) * a.n_blocks;
+    }
     if constexpr (C::PAIR_LIST) {
         // the pair tiles are found on the device: between M/256 and M/128 of them per column block;
         // the grid is sized for the most
@@ -466,11 +485,16 @@ int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_
     const int es = bf16 ? 2 : 1;
     const int64_t row_elems = C::kind == Kind::FP4 ? a.K / 2 : a.K;
     CUtensorMap ta, tb, tsa, tsb;
+    if constexpr (C::MT) {
+        BSP_TRY(operand_map_3d(&ta, o.B, a.K, a.N, o.groups, C::BM));          // B_g: 128 rows per CTA
+        BSP_TRY(operand_map(&tb, dt, es, o.A, row_elems, a.M, o.lda, C::BN_CTA));  // rows of A
+    } else {
     BSP_TRY(operand_map(&ta, dt, es, o.A, row_elems, a.M, o.lda, C::BM));
     if constexpr (C::GROUPED)
         BSP_TRY(operand_map_3d(&tb, o.B, a.K, a.N, o.groups, C::BN_CTA));
     else
         BSP_TRY(operand_map(&tb, dt, es, o.B, row_elems, a.N, o.ldb, C::BN_CTA));
+    }
     TailPlan p;
     int max_workers = 0;
     BSP_TRY(plan_gemm<C>(a, ctx, &p, &max_workers));
@@ -496,9 +520,15 @@ int launch_gemm(const Operands& o, GemmArgs a, const DeviceCtx& ctx, cudaStream_
     if constexpr (C::SCALED) {
         char* wa = base;
         char* wb = wa + ScaleChunks<C>(o, a).a_bytes;
-        rc = launch_sf_layout(o.sfa, la, wa, o.sfb, lb, wb, count, tail_bytes ? tail_count_bytes<C>(p) : 0, stream);
-        if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1);
-        if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1);
+        rc = launch_sf_layout(C::MT ? o.sfb : o.sfa, la, wa, C::MT ? o.sfa : o.sfb, lb, wb, count,
+                              tail_bytes ? tail_count_bytes<C>(p) : 0, stream);
+        if constexpr (C::MT) {
+            if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, -o.groups);
+            if (rc == BSP_OK) rc = chunk_map(&tsb, wb, 512 * C::UT_WORDS, lb.tiles, lb.q, 1);
+        } else {
+            if (rc == BSP_OK) rc = chunk_map(&tsa, wa, C::SFA_CHUNK, la.tiles, la.q, 1);
+            if (rc == BSP_OK) rc = chunk_map(&tsb, wb, C::SFB_CHUNK, lb.tiles, lb.q, C::GROUPED ? -o.groups : 1);
+        }
     } else {
         tsa = ta, tsb = tb;  // not read
         if (tail_bytes && cudaMemsetAsync(count, 0, (size_t)tail_count_bytes<C>(p), stream) != cudaSuccess)
@@ -757,7 +787,7 @@ int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, 
     a.G = G;
     a.masked_m = masked_m, a.max_m = max_m;
     a.sfb_gran = sfb_gran_n;
-    return launch_gemm<CfgMasked>(o, a, *ctx, static_cast<cudaStream_t>(stream));
+    return launch_gemm<CfgMaskedT>(o, a, *ctx, static_cast<cudaStream_t>(stream));
 }
 
 int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in, void* sf_out, int64_t ld_out,
@@ -810,7 +840,7 @@ uint64_t bsp_set_wait_timeout_ns(uint64_t ns) { return g_timeout_ns.exchange(ns)
 uint64_t bsp_kernel_launches(void) { return g_launches.load(); }
 
 int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
-    if (!plan || M <= 0 || N <= 0 || K <= 0 || kind < 0 || kind > 3) return BSP_ERR_ARG;
+    if (!plan || M <= 0 || N <= 0 || K <= 0 || kind < 0 || kind > 4) return BSP_ERR_ARG;
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
     switch (kind) {
@@ -847,6 +877,12 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                     return BSP_OK;
                 }
             }
+        case 4: {  // masked: M = rows per expert slab; work items counted for a single expert
+            BSP_TRY(describe_plan<CfgMaskedT>(M, N, K, *ctx, plan));
+            plan[4] = ((M + CfgMaskedT::MCHUNK - 1) / CfgMaskedT::MCHUNK) * ((N + CfgMaskedT::BN - 1) / CfgMaskedT::BN);
+            plan[6] = 1;
+            return BSP_OK;
+        }
         default:
             if (M / 128 <= CfgGroupedPair::MAX_PAIR_TILES)
                 return grouped_wide(N) ? describe_plan<CfgGroupedPair256>(M, N, K, *ctx, plan)

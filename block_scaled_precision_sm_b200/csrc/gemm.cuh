@@ -104,7 +104,7 @@ struct GemmCfg {
     // the first masked_m[g] (a device array) are computed; the tile list is built on the device
     static constexpr bool MASKED = MASKED_;
     static constexpr int MAX_MASKED_G = 1024;
-    static_assert(!MASKED || (GROUPED && !PAIR_), "masked layout: single-CTA grouped configs only");
+    static_assert(!MASKED || (GROUPED && (!PAIR_ || TRANS_D_)), "masked layout: single CTAs, or transposed pairs");
     // contiguous grouped layout on CTA pairs: a pair tile is one or two consecutive 128-row blocks
     // of one expert (an expert's odd last block alone, its peer CTA's rows then not stored); the
     // list of pair tiles is built on the device at kernel start from the blocks' expert indices
@@ -114,7 +114,13 @@ struct GemmCfg {
     // writes each accumulator element (row i, column j) to D[j][i]: small-M problems put the
     // long N dimension on the 256-row pair tiles
     static constexpr bool TRANS_D = TRANS_D_;
-    static_assert(!TRANS_D || !GROUPED, "transposed output: dense configs only");
+    static_assert(!TRANS_D || !GROUPED || MASKED, "transposed output: dense or masked configs only");
+    // masked layout, transposed: per expert, D_g^T = B_g A_g^T on CTA-pair tiles of 256 rows of
+    // B_g, the expert's rows of A (a chunk of up to BN of them) as the MMA's N, which is cut to
+    // the chunk's valid rows (a multiple of 16) at run time; B_g is streamed once per chunk
+    static constexpr bool MT = MASKED && TRANS_D;
+    static_assert(!MT || (PAIR_ && ACC_BUFS_ == 1 && BLOCK_N_ == 256 && KIND == Kind::FP8), "masked transposed");
+    static constexpr int MCHUNK = MT ? BN : BM;  // rows of an expert per masked work item
     // a tile's two K halves on the two CTA pairs of one 4-CTA cluster: pair 1 hands its fp32 sums
     // to pair 0 through distributed shared memory (one tile per cluster, transposed output)
     static constexpr bool CSPLIT = CSPLIT_;
@@ -215,9 +221,11 @@ __device__ __forceinline__ Work half_work(const GemmArgs& a, int w, int half, in
     return half == 0 ? Work{w, 0, mid, -1, 0} : Work{w, mid, a.num_kb, -1, 1};
 }
 
-// Masked layout: work item w is n-block w % n_blocks of the (w / n_blocks)-th valid 128-row
-// block, counting the valid blocks of expert 0 first; mprefix[g] holds the valid blocks before
-// expert g.  Returns the block's first row (in the flattened [G * max_m] rows) and its expert.
+// Masked layout: work item w is n-block w % n_blocks of the (w / n_blocks)-th valid chunk of
+// `chunk` rows, counting the valid chunks of expert 0 first; mprefix[g] holds the valid chunks
+// before expert g.  Returns the chunk's first row (in the flattened [G * max_m] rows) and its
+// expert.
+template <int CHUNK>
 __device__ __forceinline__ void masked_tile(const GemmArgs& a, const int* mprefix, int w, int* m0, int* n_blk,
                                             int* g) {
     const int mbi = w / a.n_blocks;
@@ -231,8 +239,15 @@ __device__ __forceinline__ void masked_tile(const GemmArgs& a, const int* mprefi
             lo = mid + 1;
     }
     *g = lo;
-    *m0 = lo * a.max_m + (mbi - mprefix[lo]) * 128;
+    *m0 = lo * a.max_m + (mbi - mprefix[lo]) * CHUNK;
 }
+
+// Masked transposed tile: valid rows of the chunk at flattened row m0 of expert g, and the MMA's
+// N for them (a multiple of 16, at most 256).
+__device__ __forceinline__ int masked_rows(const GemmArgs& a, const int* mcount, int g, int m0) {
+    return mcount[g] - (m0 - g * a.max_m);
+}
+__device__ __forceinline__ int masked_n(int rows) { return rows >= 256 ? 256 : (rows + 15) / 16 * 16; }
 
 // Contiguous grouped layout on CTA pairs: the pair tiles, built by one warp of each CTA.  A
 // block of 128 rows belongs to the expert of its first row (e[b] = m_indices[128 b]); a run of
@@ -428,7 +443,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     int* mprefix = reinterpret_cast<int*>(smem + C::OFF_MASK);
     int* mcount = mprefix + C::MAX_MASKED_G + 1;
     if constexpr (C::MASKED) {
-        // the tile list of the masked layout: valid 128-row blocks per expert, prefix-summed by
+        // the tile list of the masked layout: valid row chunks per expert, prefix-summed by
         // one warp (each lane a run of experts, then an exclusive scan over the lanes)
         if (warp == 2) {
             const int G = args.G, per = (G + 31) / 32;
@@ -441,7 +456,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     c = c < 0 ? 0 : args.max_m;
                 }
                 mcount[i] = c;
-                local += (c + C::BM - 1) / C::BM;
+                local += (c + C::MCHUNK - 1) / C::MCHUNK;
             }
             int incl = local;
 #pragma unroll
@@ -452,7 +467,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             int run = incl - local;
             for (int i = i0; i < i1; ++i) {
                 mprefix[i] = run;
-                run += (mcount[i] + C::BM - 1) / C::BM;
+                run += (mcount[i] + C::MCHUNK - 1) / C::MCHUNK;
             }
             if (lane == 31) mprefix[G] = incl;
         }
@@ -487,7 +502,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const auto item_of = [&](int w, bool check) {
                 Item t{Work{0, 0, args.num_kb, -1, 0}, 0, 0, 0};
                 if constexpr (C::MASKED) {
-                    masked_tile(args, mprefix, w, &t.m0, &t.n_blk, &t.g);
+                    masked_tile<C::MCHUNK>(args, mprefix, w, &t.m0, &t.n_blk, &t.g);
                 } else if constexpr (C::PAIR_LIST) {
                     int b0, len;
                     pair_tile(args, plist, w, &b0, &len, &t.n_blk);
@@ -543,7 +558,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             prior_done = true;
                         }
                     };
-                    if constexpr (C::PAIR) {
+                    if constexpr (C::MT) {
+                        // A' = this CTA's 128 rows of B_g, B' = the chunk's rows of A, split between
+                        // the two CTAs at half the tile's N; scale chunks of B_g's rows, and both
+                        // 128-row atoms of the chunk's A scales
+                        const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), pairbase);
+                        const int half_n = masked_n(masked_rows(args, mcount, g, m0)) / 2;
+                        tma_load_3d_pair(sa, &tm_a, lead_full, kx, n_blk * C::TILE_M + (int)rank * C::BM, g);
+                        tma_load_2d_pair(sb, &tm_b, lead_full, kx, m0 + (int)rank * half_n);
+                        await_prior();
+                        if (sf_here) {
+                            tma_load_4d_pair(sf, &tm_sfa, lead_full, 0, n_blk * C::CTAS + (int)rank, q, g);
+                            tma_load_3d_pair(sf + C::SFA_CHUNK, &tm_sfb, lead_full, 0, m0 / 128, q);
+                            tma_load_3d_pair(sf + C::SFA_CHUNK + 512, &tm_sfb, lead_full, 0, m0 / 128 + 1, q);
+                        }
+                    } else if constexpr (C::PAIR) {
                         const uint32_t lead_full = mapa_shared(smem_u32(&full[s]), pairbase);
                         tma_load_2d_pair(sa, &tm_a, lead_full, kx, m0);
                         if constexpr (C::GROUPED)
@@ -594,6 +623,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     (C::MASKED || C::PAIR_LIST) ? Work{0, 0, args.num_kb, -1, 0}
                     : C::CSPLIT                 ? half_work(args, w, half, C::SF_PERIOD)
                                                 : work_of(args, w, C::SF_PERIOD);
+                int tile_n = C::BN;  // the MMA's N (masked transposed: the chunk's valid rows)
+                if constexpr (C::MT) {
+                    int cm0, cnb, cg;
+                    masked_tile<C::MCHUNK>(args, mprefix, w, &cm0, &cnb, &cg);
+                    tile_n = masked_n(masked_rows(args, mcount, cg, cm0));
+                }
                 const uint32_t buf = C::ACC_BUFS == 2 ? lt & 1u : 0u;
                 const uint32_t aph = C::ACC_BUFS == 2 ? (lt >> 1) & 1u : lt & 1u;
                 if (!bounded_wait<C::PAIR>(&tmem_empty[buf], aph ^ 1u, args, abort_flag)) {
@@ -658,7 +693,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                 tc_mma_f16(d_tmem, ad, bd, id, acc);
                         } else if constexpr (C::kind == Kind::FP8) {
                             const uint32_t sid = (uint32_t)(kb % 4);
-                            const uint32_t id = idesc_block_scaled(C::TILE_M, C::BN, 0u, sid, sid);
+                            const uint32_t id = idesc_block_scaled(C::TILE_M, tile_n, 0u, sid, sid);
                             if constexpr (C::PAIR)
                                 tc_mma_mxf8_pair(d_tmem, ad, bd, id, sfa_t, sfb_t, acc);
                             else
@@ -704,7 +739,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             int m0, n_blk, g = 0;
             bool mine = true;  // this CTA's rows belong to the tile (false: the peer half of a one-block pair tile)
             if constexpr (C::MASKED) {
-                masked_tile(args, mprefix, w, &m0, &n_blk, &g);
+                masked_tile<C::MCHUNK>(args, mprefix, w, &m0, &n_blk, &g);
             } else if constexpr (C::PAIR_LIST) {
                 int b0, len;
                 pair_tile(args, plist, w, &b0, &len, &n_blk);
@@ -726,10 +761,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // masked layout: only rows below the expert's count are written; a warp whose 32
             // rows are all valid stores through TMA, one with some invalid rows row by row
             bool row_valid = mine, all_valid = mine;
-            if constexpr (C::MASKED) {
+            if constexpr (C::MASKED && !C::MT) {
                 row_valid = row - g * args.max_m < mcount[g];
                 all_valid = __all_sync(0xffffffffu, row_valid);
             }
+            // masked transposed: valid rows of the chunk (D rows m0 ...), and this warp's 32
+            // columns of D (its TMEM lanes: rows of B_g)
+            const int vrows = C::MT ? masked_rows(args, mcount, g, m0) : 0;
+            const int dcol = n_blk * C::TILE_M + (int)rank * C::BM + (int)quarter * 32;
             if constexpr (C::GROUPED && !C::MASKED) {
                 if (row < args.M && mine) {
                     const int g0 = __ldg(args.m_indices + m0);
@@ -756,6 +795,38 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // one 32 x 32 block (16 packed bf16 pairs per lane) through the swizzled staging
             // buffer to D
             const auto store_block = [&](int c, const uint32_t* w16) {
+                if constexpr (C::MT) {
+                    // accumulator column 32c + j is D row m0 + 32c + j; lane l holds D column dcol + l
+                    const int j0 = c * 32;
+                    if (j0 >= vrows || dcol >= args.N) return;
+                    if (j0 + 32 <= vrows) {
+                        // a whole block: transposed into the 64-byte-swizzled staging buffer, then TMA
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        uint8_t* blk = epi + (nblk & 1u) * C::EPI_BLOCK;
+                        const uint32_t b32 = smem_u32(blk) + (lane & 7u) * 2u;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            st_shared_u16(b32 + (uint32_t)(j * 64) + (((lane >> 3) ^ (uint32_t)((j >> 1) & 3)) << 4),
+                                          (uint16_t)(w16[j >> 1] >> (16 * (j & 1))));
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_d, blk, dcol, m0 + j0);
+                            bulk_commit_group();
+                        }
+                        ++nblk;
+                    } else if (dcol + (int)lane < args.N) {
+                        // the chunk's last block, rows past the count not touched: plain stores
+                        __nv_bfloat16* col = args.D + (int64_t)(m0 + j0) * args.ldd + dcol + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (j0 + j < vrows)
+                                *reinterpret_cast<uint16_t*>(col + (int64_t)j * args.ldd) =
+                                    (uint16_t)(w16[j >> 1] >> (16 * (j & 1)));
+                    }
+                    return;
+                }
                 if constexpr (C::TRANS_D) {
                     // element (row, n0 + 32c + j) goes to D[n0 + 32c + j][row]: for each j the
                     // warp writes 32 consecutive bf16 of one row of D

@@ -260,7 +260,7 @@ def quantize_fp8(x: torch.Tensor, block_rows: int = 1, q: torch.Tensor | None = 
     return q, sf
 
 
-_PLAN_KINDS = {"bf16": 0, "fp8": 1, "fp4": 2, "grouped_fp8": 3}
+_PLAN_KINDS = {"bf16": 0, "fp8": 1, "fp4": 2, "grouped_fp8": 3, "masked_fp8": 4}
 
 
 def gemm_plan(kind: str, M: int, N: int, K: int) -> dict:

@@ -238,7 +238,8 @@ uint64_t bsp_set_wait_timeout_ns(uint64_t ns);
 /*
  * bsp_gemm_plan — how a GEMM of this kind and shape would be launched on the current
  * device, without launching it.  kind: 0 BF16, 1 FP8 (gemm_fp8_nt), 2 FP4, 3 M-grouped FP8
- * (M = M_total).  Writes eight int32 to `plan` (caller-owned host memory):
+ * (M = M_total), 4 masked M-grouped FP8 (M = max_m; plan[4] then counts the work items of one
+ * expert whose count is max_m).  Writes eight int32 to `plan` (caller-owned host memory):
  *   plan[0] rows per tile (128 single CTA, 256 CTA pair)   plan[1] columns per tile
  *   plan[2] K slices per split tile (1: no split)          plan[3] split tiles
  *   plan[4] work items (whole tiles + slices)              plan[5] persistent workers launched

@@ -105,7 +105,7 @@ def test_rejects_bad_arguments_without_gpu(lib):
 def test_plan_rejects_bad_arguments_without_gpu(lib):
     plan = (ctypes.c_int32 * 8)()
     ptr = ctypes.cast(plan, ctypes.c_void_p)
-    assert lib.bsp_gemm_plan(4, 256, 256, 256, ptr) == -1  # no such kind
+    assert lib.bsp_gemm_plan(5, 256, 256, 256, ptr) == -1  # no such kind
     assert lib.bsp_gemm_plan(-1, 256, 256, 256, ptr) == -1
     assert lib.bsp_gemm_plan(1, 0, 256, 256, ptr) == -1
     assert lib.bsp_gemm_plan(1, 256, 256, -128, ptr) == -1

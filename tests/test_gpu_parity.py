@@ -493,6 +493,21 @@ def test_masked(ops, orc, counts, n, k):
     _check_masked(orc, p, D, f"masked {counts}")
 
 
+# Transposed masked tiles: an expert's rows in chunks of up to 256 as the MMA's N, cut to the
+# chunk's valid rows rounded up to 16 (counts on and off those boundaries, several chunks per
+# expert, a ragged N, one and two 128-row atoms of A's scales per chunk).
+@pytest.mark.parametrize("counts,max_m,n,k", [([0, 1, 16, 17, 255, 256, 257, 300, 512], 512, 1000, 512),
+                                             ([129, 128, 3], 128, 704, 1024), ([200, 64], 384, 256, 256)])
+def test_masked_transposed_chunks(ops, orc, counts, max_m, n, k):
+    plan = ops.gemm_plan("masked_fp8", max_m, n, k)
+    assert plan["transposed"] == 1 and plan["tile_m"] == 256 and plan["tile_n"] == 256, plan
+    counts = [min(c, max_m) for c in counts]
+    p = inputs.masked_fp8_problem(len(counts), max_m, n, k, seed=sum(counts), counts=counts)
+    D = _masked(ops, p)
+    _status_ok(ops)
+    _check_masked(orc, p, D, f"masked transposed {counts} max_m {max_m}")
+
+
 def test_masked_random_counts(ops, orc):
     p = inputs.masked_fp8_problem(16, 384, 640, 768, seed=77)
     D = _masked(ops, p)
