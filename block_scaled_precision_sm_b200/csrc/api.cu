@@ -259,7 +259,6 @@ using CfgGrouped = GemmCfg<Kind::FP8, 224, 4, true, false>;
 // block count fits the kernel's on-device tile list; CfgGrouped (single CTAs) otherwise
 using CfgGroupedPair = GemmCfg<Kind::FP8, 224, 6, true, true>;
 using CfgGroupedPair256 = GemmCfg<Kind::FP8, 256, 6, true, true, 1>;
-using CfgMasked = GemmCfg<Kind::FP8, 224, 4, true, false, 2, true>;
 // masked layout, transposed: 256 rows of an expert's B on a CTA pair against up to 256 of its
 // rows of A as the MMA's N (cut to the valid rows at run time), so B is streamed once per expert
 // (per 256 valid rows) instead of once per 128-row block
@@ -766,7 +765,7 @@ int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, 
                                  int64_t ld_sfb, int sfb_gran_n, void* stream) {
     if (!A || !sfa || !B || !sfb || !D || !masked_m || G < 1 || max_m <= 0 || N <= 0 || K <= 0) return BSP_ERR_ARG;
     if (sfb_gran_n != 1 && sfb_gran_n != 128) return BSP_ERR_ARG;
-    if (G > CfgMasked::MAX_MASKED_G) return BSP_ERR_UNSUPPORTED;
+    if (G > CfgMaskedT::MAX_MASKED_G) return BSP_ERR_UNSUPPORTED;
     if (K % 128 || max_m % 128) return BSP_ERR_SHAPE;
     if ((int64_t)G * max_m > 0x7fffffff) return BSP_ERR_UNSUPPORTED;
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned16(sfb)) return BSP_ERR_ALIGN;
