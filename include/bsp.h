@@ -31,8 +31,8 @@
  *     read as data nor written); K has the per-call rule stated below.
  *   - The GEMM calls take their own scratch (the scale layout for the tensor cores, the
  *     partial sums of a split last wave) stream-ordered from a pool the library keeps per
- *     device, and free it on the same stream.  Every call can be captured in a CUDA graph;
- *     under capture the scratch becomes a graph memory node.
+ *     device, and free it on the same stream.  These calls can be captured in a CUDA
+ *     graph; under capture the scratch becomes a graph memory node.
  *   - Results are deterministic: the same inputs give the same bytes on every run.
  *
  * Packed scale-factor layout ("SF words"): for a matrix with MN scale rows and KB scale
