@@ -274,6 +274,8 @@ using CfgFP4S = GemmCfg<Kind::FP4, 128, 7, false, true, 2, false, true>;
 // run on the two CTA pairs of a 4-CTA cluster and meet in distributed shared memory instead of
 // a global workspace (one tile per cluster)
 using CfgFP8S2 = GemmCfg<Kind::FP8, 128, 8, false, true, 2, false, true, true>;
+using CfgBF16S2 = GemmCfg<Kind::BF16, 128, 8, false, true, 2, false, true, true>;
+using CfgFP4S2 = GemmCfg<Kind::FP4, 128, 7, false, true, 2, false, true, true>;
 
 // Grouped pair tiles 256 columns wide unless 224-wide ones cover N with enough fewer wasted
 // columns to make up for being about 8% less efficient.
@@ -661,6 +663,7 @@ int gemm_bf16_nt(const void* A, const void* B, void* D, int M, int N, int K, int
         default: {  // Swap: M <= 128
             Operands os = o;
             swap_operands(os, a);
+            if (use_cluster_split<CfgBF16S, CfgBF16S2>(a, *ctx)) return launch_gemm<CfgBF16S2>(os, a, *ctx, st);
             return launch_gemm<CfgBF16S>(os, a, *ctx, st);
         }
     }
@@ -725,6 +728,7 @@ int gemm_fp4_nt(const void* A, const void* sfa, const void* B, const void* sfb, 
         default: {  // Swap: M <= 128
             Operands os = o;
             swap_operands(os, a);
+            if (use_cluster_split<CfgFP4S, CfgFP4S2>(a, *ctx)) return launch_gemm<CfgFP4S2>(os, a, *ctx, st);
             return launch_gemm<CfgFP4S>(os, a, *ctx, st);
         }
     }
@@ -850,6 +854,9 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                 default: {  // Swap: M <= 128
                     BSP_TRY(describe_plan<CfgBF16S>(N, M, K, *ctx, plan));
                     plan[6] = 1;
+                    GemmArgs t{};
+                    t.M = N, t.N = M, t.K = K;
+                    plan[7] = use_cluster_split<CfgBF16S, CfgBF16S2>(t, *ctx) ? 1 : 0;
                     return BSP_OK;
                 }
             }
@@ -873,6 +880,9 @@ int bsp_gemm_plan(int kind, int M, int N, int K, int32_t* plan) {
                 default: {  // Swap: M <= 128
                     BSP_TRY(describe_plan<CfgFP4S>(N, M, K, *ctx, plan));
                     plan[6] = 1;
+                    GemmArgs t{};
+                    t.M = N, t.N = M, t.K = K;
+                    plan[7] = use_cluster_split<CfgFP4S, CfgFP4S2>(t, *ctx) ? 1 : 0;
                     return BSP_OK;
                 }
             }

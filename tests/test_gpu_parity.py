@@ -247,6 +247,18 @@ def test_fp8_small_m_cluster_split(ops, orc, m, n, k, gran):
     assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
 
 
+# The same cluster split for BF16 and FP4 (FP4 carrying its scale chunks every K step)
+@pytest.mark.parametrize("kind,m,n,k", [("bf16", 64, 7000, 1024), ("bf16", 128, 6500, 2048), ("fp4", 40, 6500, 4096),
+                                        ("fp4", 128, 7168, 4096)])
+def test_bf16_fp4_small_m_cluster_split(ops, orc, kind, m, n, k):
+    plan = ops.gemm_plan(kind, m, n, k)
+    assert plan["cluster_split"] == 1 and plan["splits"] == 2 and plan["transposed"] == 1, plan
+    got, ref = _run_kind(ops, kind, m, n, k, seed=m + n + k)
+    check_gemm(got, ref(orc), f"{kind} cluster split {m}x{n}x{k}")
+    again, _ = _run_kind(ops, kind, m, n, k, seed=m + n + k)
+    assert np.array_equal(got, again)
+
+
 @pytest.mark.parametrize("kind,m,n,k", [("bf16", 128, 3000, 2048), ("bf16", 5, 448, 640), ("fp4", 128, 2000, 4096),
                                         ("fp4", 40, 704, 1024)])
 def test_bf16_fp4_small_m_run_transposed(ops, orc, kind, m, n, k):
