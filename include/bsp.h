@@ -246,8 +246,9 @@ uint64_t bsp_set_wait_timeout_ns(uint64_t ns);
  *   plan[6] 1 if the product is computed transposed, D^T = B A^T (M <= 128: the tile rows
  *           then run along N and the columns along M), else 0
  *   plan[7] 1 if the two K slices of every tile run on the two CTA pairs of one 4-CTA cluster
- *           and are added in distributed shared memory (FP8, M <= 128, two slices per tile,
- *           all tiles co-resident), else 0; the sums and their order are the same either way
+ *           and are added in distributed shared memory (BF16, FP8 or FP4 at M <= 128, two slices
+ *           per tile, all tiles co-resident), else 0; the sums and their order are the same
+ *           either way
  * The tiles left after the last full wave of workers are cut along K into slices at
  * scale-group boundaries when that shortens the last wave (at least two slices of eight or
  * more K steps); their fp32 partial sums meet in a workspace and are added in slice order
