@@ -68,6 +68,10 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     const int rn = min(kSfTileMN, mn - r0);         // input rows in this tile (<= 0: padding only)
     const int vpr = (kn + EV - 1) / EV;             // loads per row
     const int total = rn > 0 ? rn * vpr : 0;
+    // idx / vpr as a multiply-high by ceil(2^32 / vpr): exact for idx < 2^13 and 2 <= vpr <= 64
+    // (vpr = 1 is idx itself)
+    const uint32_t vrec = vpr > 1 ? (uint32_t)((0x100000000ull + (uint64_t)vpr - 1) / (uint64_t)vpr) : 0u;
+    const auto row_of = [&](int idx) { return vpr > 1 ? (int)__umulhi((uint32_t)idx, vrec) : idx; };
     const int t = threadIdx.x;
     bool bad = false;
 
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     for (int it = 0; it < MAX_VECS; ++it) {
         const int idx = t + it * kSfThreads;
         if (idx < total) {
-            const int i = idx / vpr, k = (idx - i * vpr) * EV;
+            const int i = row_of(idx), k = (idx - i * vpr) * EV;
             const char* src = static_cast<const char*>(in) + ((int64_t)(r0 + i) * ld_in + k0 + k) * ES;
             if (k + EV <= kn) {
                 v[it] = __ldg(reinterpret_cast<const V*>(src));
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     for (int it = 0; it < MAX_VECS; ++it) {
         const int idx = t + it * kSfThreads;
         if (idx < total) {
-            const int i = idx / vpr, k = (idx - i * vpr) * EV;
+            const int i = row_of(idx), k = (idx - i * vpr) * EV;
 #pragma unroll
             for (int e = 0; e < EV; ++e) {
                 if (k + e < kn) {
