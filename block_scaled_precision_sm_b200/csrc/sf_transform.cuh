@@ -57,7 +57,11 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     constexpr int ES = IN_KIND == 0 ? 4 : 1;       // input element bytes
     constexpr int EV = VEC / ES;                   // elements per load
     static_assert(EV >= 1 && kSfTileKB % EV == 0, "vector width");
-    constexpr int MAX_VECS = kSfTileMN * (kSfTileKB / EV) / kSfThreads;  // loads per thread, at most
+    // Loads go in groups of four rows at one K vector ("quads"): a thread's four loads are the same
+    // K range of four consecutive rows, so each K block's four exponent bytes become one 32-bit
+    // shared-memory store.  Consecutive threads take consecutive vectors of a row (coalesced).
+    constexpr int RQ = 4;
+    constexpr int MAX_Q = (kSfTileMN / RQ * (kSfTileKB / EV) + kSfThreads - 1) / kSfThreads;  // quads per thread
     constexpr int PITCH = kSfTileMN + 16;          // bytes per K block in shared memory
     using V = typename SfVec<VEC>::T;
     __shared__ __align__(16) uint8_t eT[kSfTileKB][PITCH];
@@ -67,67 +71,79 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     const int kn = min(kSfTileKB, kb - k0);         // scale blocks in this tile
     const int rn = min(kSfTileMN, mn - r0);         // input rows in this tile (<= 0: padding only)
     const int vpr = (kn + EV - 1) / EV;             // loads per row
-    const int total = rn > 0 ? rn * vpr : 0;
-    // idx / vpr as a multiply-high by ceil(2^32 / vpr): exact for idx < 2^13 and 2 <= vpr <= 64
-    // (vpr = 1 is idx itself)
+    const int quads = rn > 0 ? ((rn + RQ - 1) / RQ) * vpr : 0;
+    // qidx / vpr as a multiply-high by ceil(2^32 / vpr): exact for qidx < 2^13 and 2 <= vpr <= 64
+    // (vpr = 1 is qidx itself)
     const uint32_t vrec = vpr > 1 ? (uint32_t)((0x100000000ull + (uint64_t)vpr - 1) / (uint64_t)vpr) : 0u;
-    const auto row_of = [&](int idx) { return vpr > 1 ? (int)__umulhi((uint32_t)idx, vrec) : idx; };
+    const auto group_of = [&](int qidx) { return vpr > 1 ? (int)__umulhi((uint32_t)qidx, vrec) : qidx; };
     const int t = threadIdx.x;
     bool bad = false;
 
-    // all loads first (up to MAX_VECS in flight per thread), then the bytes into shared memory
-    V v[MAX_VECS];
+    // all loads first (up to MAX_Q quads in flight per thread), then the bytes into shared memory
+    V v[MAX_Q][RQ];
 #pragma unroll
-    for (int it = 0; it < MAX_VECS; ++it) {
-        const int idx = t + it * kSfThreads;
-        if (idx < total) {
-            const int i = row_of(idx), k = (idx - i * vpr) * EV;
-            const char* src = static_cast<const char*>(in) + ((int64_t)(r0 + i) * ld_in + k0 + k) * ES;
-            if (k + EV <= kn) {
-                v[it] = __ldg(reinterpret_cast<const V*>(src));
-            } else {  // a partial vector at the end of a row: the elements that exist, zeros after
-                uint32_t w[VEC >= 4 ? VEC / 4 : 1] = {};
+    for (int it = 0; it < MAX_Q; ++it) {
+        const int qidx = t + it * kSfThreads;
+        if (qidx < quads) {
+            const int g = group_of(qidx), k = (qidx - g * vpr) * EV;
 #pragma unroll
-                for (int e = 0; e < EV; ++e) {
-                    if (k + e < kn) {
-                        const uint32_t x = ES == 4 ? __ldg(reinterpret_cast<const uint32_t*>(src) + e)
-                                                   : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(src) + e);
-                        if (ES == 4)
-                            w[e] = x;
-                        else
-                            w[e / 4] |= x << (8 * (e % 4));
+            for (int q = 0; q < RQ; ++q) {
+                const int i = RQ * g + q;
+                const char* src = static_cast<const char*>(in) + ((int64_t)(r0 + i) * ld_in + k0 + k) * ES;
+                if (i < rn && k + EV <= kn) {
+                    v[it][q] = __ldg(reinterpret_cast<const V*>(src));
+                } else {  // a row past the tile's, or a partial vector at the end of a row: zeros after
+                    uint32_t w[VEC >= 4 ? VEC / 4 : 1] = {};
+                    if (i < rn) {
+#pragma unroll
+                        for (int e = 0; e < EV; ++e) {
+                            if (k + e < kn) {
+                                const uint32_t x = ES == 4 ? __ldg(reinterpret_cast<const uint32_t*>(src) + e)
+                                                           : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(src) + e);
+                                if (ES == 4)
+                                    w[e] = x;
+                                else
+                                    w[e / 4] |= x << (8 * (e % 4));
+                            }
+                        }
                     }
+                    if constexpr (VEC == 16)
+                        v[it][q] = make_uint4(w[0], w[1], w[2], w[3]);
+                    else if constexpr (VEC == 8)
+                        v[it][q] = make_uint2(w[0], w[1]);
+                    else if constexpr (VEC == 4)
+                        v[it][q] = w[0];
+                    else
+                        v[it][q] = (uint8_t)w[0];
                 }
-                if constexpr (VEC == 16)
-                    v[it] = make_uint4(w[0], w[1], w[2], w[3]);
-                else if constexpr (VEC == 8)
-                    v[it] = make_uint2(w[0], w[1]);
-                else if constexpr (VEC == 4)
-                    v[it] = w[0];
-                else
-                    v[it] = (uint8_t)w[0];
             }
         }
     }
 #pragma unroll
-    for (int it = 0; it < MAX_VECS; ++it) {
-        const int idx = t + it * kSfThreads;
-        if (idx < total) {
-            const int i = row_of(idx), k = (idx - i * vpr) * EV;
+    for (int it = 0; it < MAX_Q; ++it) {
+        const int qidx = t + it * kSfThreads;
+        if (qidx < quads) {
+            const int g = group_of(qidx), k = (qidx - g * vpr) * EV;
 #pragma unroll
             for (int e = 0; e < EV; ++e) {
                 if (k + e < kn) {
-                    uint32_t b;
-                    if constexpr (IN_KIND == 0) {
-                        const uint32_t bits = SfVec<VEC>::word(v[it], e);
-                        b = (bits >> 23) & 0xFFu;
-                        // an exact positive normal power of two: sign 0, mantissa 0, exponent 1..254
-                        bad |= (bits & 0x807FFFFFu) != 0u || b == 0u || b == 255u;
-                    } else {
-                        b = (SfVec<VEC>::word(v[it], e / 4) >> (8 * (e % 4))) & 0xFFu;
-                        bad |= b == 255u;  // UE8M0 0xFF is NaN
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int q = 0; q < RQ; ++q) {
+                        uint32_t b;
+                        if constexpr (IN_KIND == 0) {
+                            const uint32_t bits = SfVec<VEC>::word(v[it][q], e);
+                            b = (bits >> 23) & 0xFFu;
+                            // an exact positive normal power of two: sign 0, mantissa 0, exponent 1..254
+                            // (rows past the tile's hold 0 and are not checked)
+                            if (RQ * g + q < rn) bad |= (bits & 0x807FFFFFu) != 0u || b == 0u || b == 255u;
+                        } else {
+                            b = (SfVec<VEC>::word(v[it][q], e / 4) >> (8 * (e % 4))) & 0xFFu;
+                            bad |= b == 255u;  // UE8M0 0xFF is NaN
+                        }
+                        word |= b << (8 * q);
                     }
-                    eT[k + e][i] = (uint8_t)b;
+                    *reinterpret_cast<uint32_t*>(&eT[k + e][RQ * g]) = word;
                 }
             }
         }
