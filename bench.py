@@ -601,12 +601,16 @@ def secondary(torch, ops, timer, args, peaks, peak_kind, sampler, sms):
     out[k] = v
     del pm, dm, sfa_m, sfb_m, Dm
 
-    # scale transform alone: config-3 SFA (fp32 scales [M_total, 56]) -> int16 words, and the same
-    # rows 64 times over in one call (where bandwidth rather than launch latency bounds it)
+    # scale transform alone: the grouped workload's SFA (fp32 scales [M_total, 56]) -> int16 words,
+    # the same rows 64 times over in one call (where bandwidth rather than launch latency bounds
+    # it), and the FP4 workload's B scales (fp32, one per 32 K: [7168, 512])
     s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()
     del g, dg, Dg
-    for name, src in (("sf_transform_fp32_36864x56", s32), ("sf_transform_fp32_64x36864x56", s32.repeat(64, 1))):
-        w = torch.empty((28, ops.sf_ld(src.shape[0])), dtype=torch.int16, device="cuda")
+    e4 = np.random.default_rng(44).integers(110, 140, size=(N, K // 32)).astype(np.int32)
+    s4 = torch.from_numpy(np.ldexp(np.float32(1), e4 - 127).astype(np.float32)).cuda()
+    for name, src in (("sf_transform_fp32_36864x56", s32), ("sf_transform_fp32_64x36864x56", s32.repeat(64, 1)),
+                      ("sf_transform_fp32_7168x512", s4)):
+        w = torch.empty(((src.shape[1] + 1) // 2, ops.sf_ld(src.shape[0])), dtype=torch.int16, device="cuda")
         spans, clk = timed(one_call(lambda src=src, w=w: ops.transform_sf_ue8m0(src, out=w)))
         ms = float(np.mean(spans))
         moved = src.numel() * 4 + w.numel() * 2
@@ -615,7 +619,7 @@ def secondary(torch, ops, timer, args, peaks, peak_kind, sampler, sms):
                      "frac": round(moved / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                      "traffic": profiled_traffic(name + ".md"), "sm_mhz": clk.get("sm_mhz")}
         del w
-    del s32
+    del s32, s4
 
     # the quantiser (the step before the GEMM): the headline's A as fp32 in 1x128 blocks and its
     # B as bf16 in 128x128 blocks, values -> E4M3 codes + packed UE8M0 words
@@ -666,7 +670,8 @@ def run_reference(args):
 
     oracle.build()
     p = inputs.dense_fp8_problem(M, N, K, seed=100)
-    rows_per_step = 2
+    # 32 rows a step (about 0.1-0.2 s on the machine's cores): enough rows for every host thread
+    rows_per_step = 32
 
     def step(i):
         r0 = (i * rows_per_step) % M
