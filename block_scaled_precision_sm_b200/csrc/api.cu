@@ -365,16 +365,25 @@ int launch_sf_layout(const void* in_a, const SfLayout& pa, void* out_a, const vo
                      void* out_b, void* zero, int64_t zero_bytes, cudaStream_t stream) {
     const int64_t total = sf_layout_words(pa) + sf_layout_words(pb) + zero_bytes / 16;
     const int64_t blocks = (total + 255) / 256;
-    // a grid that is resident at once (grid-stride loop): every CTA reaches the early
-    // launch_dependents right away, so the GEMM after it is launched without waiting
+    // a grid that is resident at once (grid-stride loop): every CTA reaches launch_dependents as
+    // soon as the kernel before it has completed, so the GEMM after it launches at that moment
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t cap = (int64_t)sms * 4;
-    sf_tmem_layout_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(
-        static_cast<const uint16_t*>(in_a), pa, static_cast<uint32_t*>(out_a), static_cast<const uint16_t*>(in_b),
-        pb, static_cast<uint32_t*>(out_b), static_cast<uint4*>(zero), zero_bytes / 16);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, sf_tmem_layout_kernel, static_cast<const uint16_t*>(in_a), pa,
+                                             static_cast<uint32_t*>(out_a), static_cast<const uint16_t*>(in_b), pb,
+                                             static_cast<uint32_t*>(out_b), static_cast<uint4*>(zero), zero_bytes / 16);
     g_launches.fetch_add(1);
-    return cudaGetLastError() == cudaSuccess ? BSP_OK : BSP_ERR_CUDA;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? BSP_OK : BSP_ERR_CUDA;
 }
 
 // Stream-ordered scratch from a pool this library owns on each device, which keeps its memory

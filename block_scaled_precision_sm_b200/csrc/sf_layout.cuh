@@ -70,8 +70,11 @@ __global__ void __launch_bounds__(256) sf_tmem_layout_kernel(const uint16_t* __r
                                                              const uint16_t* __restrict__ in_b, SfLayout pb,
                                                              uint32_t* __restrict__ out_b, uint4* __restrict__ zero,
                                                              int64_t zero_vecs) {
-    // the GEMM that follows may start its set-up and operand loads now; it waits for this
-    // kernel's writes before it reads them
+    // Launched with programmatic stream serialisation: wait for the kernel before this one (the
+    // scale transforms, typically), then let the GEMM that follows start its set-up and operand
+    // loads; it waits for this kernel's writes before it reads them.  Triggering only after the
+    // wait means the GEMM starts after every kernel ahead of this one has completed.
+    griddep_wait();
     griddep_launch_dependents();
     const int64_t na = sf_layout_words(pa), nab = na + sf_layout_words(pb), total = nab + zero_vecs;
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;

@@ -16,6 +16,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace bsp {
 
 constexpr int kSfTileMN = 128;  // rows per CTA
@@ -78,6 +80,21 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     const auto group_of = [&](int qidx) { return vpr > 1 ? (int)__umulhi((uint32_t)qidx, vrec) : qidx; };
     const int t = threadIdx.x;
     bool bad = false;
+
+    // The kernel is launched with programmatic stream serialisation, so it may start while the
+    // kernel before it still runs.  Until that one has completed it only brings its own input
+    // rows into L2 (every prefetched address is a byte read below); then it waits, and only then
+    // lets the next kernel launch, so whatever follows starts after everything before this one.
+    {
+        constexpr int LPR = (kSfTileKB * ES + 127) / 128 + 1;  // prefetch points per row
+        const int bytes = kn * ES;
+        for (int i = t; i < max(rn, 0) * LPR; i += kSfThreads) {
+            const int row = i / LPR, l = i - row * LPR;
+            prefetch_l2(static_cast<const char*>(in) + ((int64_t)(r0 + row) * ld_in + k0) * ES + min(l * 128, bytes - 1));
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
 
     // all loads first (up to MAX_Q quads in flight per thread), then the bytes into shared memory
     V v[MAX_Q][RQ];
@@ -179,30 +196,40 @@ inline int sf_transform_vec(const void* in, int in_kind, int64_t ld_in) {
     return es == 4 ? 4 : 1;
 }
 
-// Launch on `stream`; false if the launch failed or the grid is too large.
+template <int IN_KIND, int VEC>
+inline bool launch_sf_transform_vec(dim3 grid, const void* in, int mn, int kb, int64_t ld_in, uint16_t* out,
+                                    int64_t ld_out, int* status, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kSfThreads);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, sf_transform_kernel<IN_KIND, VEC>, in, mn, kb, ld_in, out, ld_out, status) ==
+           cudaSuccess;
+}
+
+// Launch on `stream` (programmatic serialisation: the kernel waits for the one before it);
+// false if the launch failed or the grid is too large.
 inline bool launch_sf_transform(const void* in, int in_kind, int mn, int kb, int64_t ld_in, uint16_t* out,
                                 int64_t ld_out, int* status, cudaStream_t stream) {
     const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
     if (grid.y > 65535u) return false;
     const int vec = sf_transform_vec(in, in_kind, ld_in);
-    if (in_kind == 0) {
-        if (vec == 16)
-            sf_transform_kernel<0, 16><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-        else if (vec == 8)
-            sf_transform_kernel<0, 8><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-        else
-            sf_transform_kernel<0, 4><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-    } else {
-        if (vec == 16)
-            sf_transform_kernel<1, 16><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-        else if (vec == 8)
-            sf_transform_kernel<1, 8><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-        else if (vec == 4)
-            sf_transform_kernel<1, 4><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-        else
-            sf_transform_kernel<1, 1><<<grid, kSfThreads, 0, stream>>>(in, mn, kb, ld_in, out, ld_out, status);
-    }
-    return cudaGetLastError() == cudaSuccess;
+    bool ok;
+    if (in_kind == 0)
+        ok = vec == 16  ? launch_sf_transform_vec<0, 16>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<0, 8>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
+                        : launch_sf_transform_vec<0, 4>(grid, in, mn, kb, ld_in, out, ld_out, status, stream);
+    else
+        ok = vec == 16  ? launch_sf_transform_vec<1, 16>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<1, 8>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
+             : vec == 4 ? launch_sf_transform_vec<1, 4>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
+                        : launch_sf_transform_vec<1, 1>(grid, in, mn, kb, ld_in, out, ld_out, status, stream);
+    return ok && cudaGetLastError() == cudaSuccess;
 }
 
 }  // namespace bsp
