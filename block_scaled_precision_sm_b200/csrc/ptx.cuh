@@ -109,9 +109,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Brings the 128-byte line that holds `p` into L2; nothing waits for it.
-__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-
 // Orders this thread's async-proxy global accesses (completed bulk copies) with its later
 // generic-proxy ones.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -82,17 +82,9 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __
     bool bad = false;
 
     // The kernel is launched with programmatic stream serialisation, so it may start while the
-    // kernel before it still runs.  Until that one has completed it only brings its own input
-    // rows into L2 (every prefetched address is a byte read below); then it waits, and only then
-    // lets the next kernel launch, so whatever follows starts after everything before this one.
-    {
-        constexpr int LPR = (kSfTileKB * ES + 127) / 128 + 1;  // prefetch points per row
-        const int bytes = kn * ES;
-        for (int i = t; i < max(rn, 0) * LPR; i += kSfThreads) {
-            const int row = i / LPR, l = i - row * LPR;
-            prefetch_l2(static_cast<const char*>(in) + ((int64_t)(r0 + row) * ld_in + k0) * ES + min(l * 128, bytes - 1));
-        }
-    }
+    // kernel before it still runs: it waits for that one before touching global memory, and only
+    // then lets the next kernel launch, so whatever follows starts after everything before this
+    // one has completed.
     griddep_wait();
     griddep_launch_dependents();
 

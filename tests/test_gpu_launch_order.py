@@ -1,16 +1,18 @@
 """Launch order: inputs written by the kernel just before a call, buffers reused call after call.
 
 The scale transform, the scale-layout pass and the GEMM are launched with programmatic stream
-serialisation, so each may start while the kernel before it still runs.  Each waits for that
-kernel before it reads what that kernel may write or writes what it may read; the GEMM reads
-its operands (and the grouped kernels their expert indices or counts) before it waits, which
-is sound only because the layout pass lets it start once every kernel ahead has completed.
-These tests put that to work: on a side stream, behind a long kernel, ordinary torch kernels
-write the operands, scales, indices or counts immediately before each call, two input sets
-alternate, the library's packed-scale buffers (or the fixed scratch of the no-allocation entry
-point) are reused by the next call, and a torch kernel copies D right after.  Every result must
-equal, bit for bit, the one computed for its input set with synchronisations around the call,
-and that one is checked against the fp64 oracle first.
+serialisation, so each may start while the kernel before it still runs (the quantiser is not,
+but the layout pass after it is).
+Each waits for that kernel before it reads what that kernel may write or writes what it may
+read; the GEMM reads its operands (and the grouped kernels their expert indices or counts)
+before it waits, which is sound only because the layout pass lets it start once every kernel
+ahead has completed.  These tests put that to work: on a side stream, behind a long kernel,
+ordinary torch kernels write the operands, scales, indices, counts or the quantiser's input
+immediately before each call, two input sets alternate, the library's packed-scale buffers (or
+the fixed scratch of the no-allocation entry point) are reused by the next call, and a torch
+kernel copies D right after.  Every result must equal, bit for bit, the one computed for its
+input set with synchronisations around the call, and that one is checked against the fp64
+oracle first.
 """
 
 import ctypes
@@ -210,3 +212,35 @@ def test_masked_counts_written_just_before_each_call(ops, orc, busy):
     assert ops.device_status() == 0
     for i, D in enumerate(outs):
         assert _same_bits(D, refs[i % 2]), f"masked, round {i}"
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 1024, 2048), (384, 672, 1024)])
+def test_quantiser_output_read_by_the_next_call(ops, orc, busy, m, n, k):
+    # quantise (fp32 activations, 1 x 128 blocks) and multiply, with nothing between the two calls
+    pb = inputs.dense_fp8_problem(m, n, k, seed=71)
+    B, sfb = to_dev(pb["B"]), ops.transform_sf_ue8m0(to_dev(pb["sfb"]))
+    xs = [inputs.normal_matrix(m, k, seed=s) for s in (72, 73)]
+    src = [to_dev(x) for x in xs]
+    refs = []
+    for x, xd in zip(xs, src):
+        torch.cuda.synchronize()
+        q, sf = ops.quantize_fp8(xd)
+        D = ops.gemm_fp8_nt(q, sf, B, sfb)
+        torch.cuda.synchronize()
+        assert ops.device_status() == 0
+        qa, ea = orc.quantize_fp8(x, 1)
+        check_gemm(bf16_to_f64(D), orc.gemm_fp8(qa, ea, pb["B"], pb["sfb"]), f"quantise + gemm {m}x{n}x{k}")
+        refs.append(D)
+    x_buf = torch.empty_like(src[0])
+    q_buf = torch.empty((m, k), dtype=torch.uint8, device="cuda")
+    sf_buf = torch.empty(((k // 128 + 1) // 2, ops.sf_ld(m)), dtype=torch.int16, device="cuda")
+    D_buf = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+
+    def call(j):
+        ops.quantize_fp8(x_buf, q=q_buf, sf=sf_buf)
+        return ops.gemm_fp8_nt(q_buf, sf_buf, B, sfb, D_buf)
+
+    outs = _run_rounds(busy, lambda j: x_buf.copy_(src[j]), call, 2)
+    assert ops.device_status() == 0
+    for i, D in enumerate(outs):
+        assert _same_bits(D, refs[i % 2]), f"quantise + gemm, round {i}"
