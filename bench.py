@@ -90,8 +90,9 @@ def parse():
                     help="none: one independent problem per GPU (weak scaling); n: one problem split along N "
                          "over the ranks (strong scaling)")
     ap.add_argument("--gather", action="store_true", help="with --shard n: all-gather D inside every step")
-    ap.add_argument("--profile", choices=["fp8", "fp8_m128", "bf16", "fp4", "grouped", "masked", "sf_transform", "sf_transform_64x",
-                                          "quantize_act", "quantize_wgt"],
+    ap.add_argument("--profile", choices=["fp8", "fp8_m128", "fp8_m1024", "fp8_m4096", "bf16", "fp4", "grouped", "masked",
+                                          "sf_transform", "sf_transform_64x", "sf_transform_fp4", "quantize_act",
+                                          "quantize_wgt"],
                     help="launch only this kernel (warm-up + steps launches, no timing) for an ncu capture")
     return ap.parse_args()
 
@@ -559,8 +560,8 @@ def secondary(torch, ops, timer, args, peaks, peak_kind, sampler, sms):
                          "hbm_gbs_min_bytes": round(bytes_min / (ms * 1e-3) / 1e9, 1),
                          "hbm_frac_min_bytes": round(bytes_min / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                          "plan": ops.gemm_plan("fp8", m, 7168, 7168), "sm_mhz": clk.get("sm_mhz")}
-        if m == 128:
-            sweep[str(m)]["traffic"] = profiled_traffic("gemm_fp8_transposed_128x7168x7168.md")
+        sweep[str(m)]["traffic"] = profiled_traffic("gemm_fp8_transposed_128x7168x7168.md" if m == 128 else
+                                                    f"gemm_fp8_{m}x7168x7168.md")
         del p, dv, sa, sb, Dm
     out["fp8_m_sweep_n7168_k7168"] = sweep
 
@@ -709,10 +710,11 @@ def run_profile(args):
         sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
         D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         fn = lambda: ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # noqa: E731
-    elif args.profile == "fp8_m128":
-        p, dv = fp8_device_problem(torch, 128, 7168, 7168, seed=30 + 128)
+    elif args.profile in ("fp8_m128", "fp8_m1024", "fp8_m4096"):  # the M sweep at N = K = 7168
+        m = int(args.profile[5:])
+        p, dv = fp8_device_problem(torch, m, 7168, 7168, seed=30 + m)
         sa, sb = ops.transform_sf_ue8m0(dv["sfa"]), ops.transform_sf_ue8m0(dv["sfb"])
-        D = torch.empty((128, 7168), dtype=torch.bfloat16, device="cuda")
+        D = torch.empty((m, 7168), dtype=torch.bfloat16, device="cuda")
         fn = lambda: ops.gemm_fp8_nt(dv["A"], sa, dv["B"], sb, D)  # noqa: E731
     elif args.profile == "bf16":
         p = inputs.dense_bf16_problem(M, N, K, seed=2)
@@ -748,6 +750,11 @@ def run_profile(args):
         br = 1 if act else 128
         qx, sx = ops.quantize_fp8(x, br)
         fn = lambda: ops.quantize_fp8(x, br, q=qx, sf=sx)  # noqa: E731
+    elif args.profile == "sf_transform_fp4":  # the FP4 workload's B scales, fp32 [7168, 512]
+        e4 = np.random.default_rng(44).integers(110, 140, size=(N, K // 32)).astype(np.int32)
+        s4 = torch.from_numpy(np.ldexp(np.float32(1), e4 - 127).astype(np.float32)).cuda()
+        w = torch.empty((K // 64, ops.sf_ld(N)), dtype=torch.int16, device="cuda")
+        fn = lambda: ops.transform_sf_ue8m0(s4, out=w)  # noqa: E731
     else:
         g = inputs.grouped_fp8_problem(32, 32768, 4096, 7168, seed=8)
         s32 = torch.from_numpy(np.ldexp(np.float32(1), g["sfa"].astype(np.int32) - 127).astype(np.float32)).cuda()
