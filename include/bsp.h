@@ -21,6 +21,11 @@
  *   - Every pointer is a DEVICE pointer owned by the caller; the library never frees
  *     or retains caller memory.  Work is enqueued asynchronously on `stream` (a
  *     cudaStream_t passed as void*; NULL = legacy default stream) on the current device.
+ *     Stream order holds as for any kernel: a call's kernels start reading and writing
+ *     memory only after the work enqueued before them on `stream` has completed.  (The
+ *     scaled GEMMs, the scale transform and the scale-layout pass are launched with
+ *     programmatic stream serialisation, so their launch and set-up may overlap the kernel
+ *     before them; each waits for it before touching memory.)
  *   - Argument errors are returned synchronously and nothing is launched.  Launch
  *     failures return BSP_ERR_CUDA.  Faults found while the kernels run (a wait that
  *     timed out, a malformed scale or expert index) are latched in a per-device status
