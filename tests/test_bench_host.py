@@ -76,3 +76,21 @@ def test_clock_window_selects_the_timed_samples(monkeypatch):
     # a window shorter than the sampling period takes the samples on either side
     assert s.window(1.5, 1.6)["samples"] == 2
     assert bench.ClockSampler(0).window()["samples"] == 0
+
+
+def test_every_profile_the_bench_reads_is_committed_with_its_figures():
+    # the summaries bench.py looks up for its traffic figures, and the ones its --profile cases write
+    import re
+
+    text = open(os.path.join(os.path.dirname(bench.__file__), "bench.py")).read()
+    names = set(re.findall(r'profiled_traffic\("([^"]+\.md)"', text))
+    names |= {"gemm_fp8_1024x7168x7168.md", "gemm_fp8_4096x7168x7168.md", "sf_transform_fp32_36864x56.md",
+              "sf_transform_fp32_64x36864x56.md", "sf_transform_fp32_7168x512.md",
+              "quantize_fp8_fp32_4096x16384_1x128.md", "quantize_fp8_bf16_7168x16384_128x128.md"}
+    for name in sorted(names):
+        path = os.path.join(bench.ROOT, "profiles", name)
+        assert os.path.exists(path), name
+        body = open(path).read()
+        assert re.search(r"traffic_bytes_per_launch:\s*[0-9]+", body), name
+        assert re.search(r"sources_digest:\s*[0-9a-f]{16}", body), name
+        assert "--clock-control none" in body and "python bench.py --profile" in body, name
