@@ -342,8 +342,7 @@ def run_ours(args):
     def step(ev):
         if ev is not None:
             ev[0].record()
-        ops.transform_sf_ue8m0(dev["sfa"], out=sfa_w)
-        ops.transform_sf_ue8m0(dev["sfb"], out=sfb_w)
+        ops.transform_sf_ue8m0_pair(dev["sfa"], dev["sfb"], out_a=sfa_w, out_b=sfb_w)  # both scale tensors
         if ev is not None:
             ev[1].record()
         ops.gemm_fp8_nt(dev["A"], sfa_w, dev["B"], sfb_w, D, sfb_gran_n=128)

@@ -589,10 +589,13 @@ int status_word(int** out) {
 
 void note_launch() { g_launches.fetch_add(1); }
 
-int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
-                           cudaStream_t stream) {
+int launch_sf_transform_u8_pair(const void* in_a, int mn_a, int64_t ld_in_a, void* out_a, int64_t ld_out_a,
+                                const void* in_b, int mn_b, int64_t ld_in_b, void* out_b, int64_t ld_out_b, int kb,
+                                int* status, cudaStream_t stream) {
     if ((kb + kSfTileKB - 1) / kSfTileKB > 65535) return BSP_ERR_UNSUPPORTED;
-    const bool ok = launch_sf_transform(in, 1, mn, kb, ld_in, static_cast<uint16_t*>(out), ld_out, status, stream);
+    const SfJob jobs[2] = {{in_a, ld_in_a, static_cast<uint16_t*>(out_a), ld_out_a, mn_a},
+                           {in_b, ld_in_b, static_cast<uint16_t*>(out_b), ld_out_b, mn_b}};
+    const bool ok = launch_sf_transform(jobs, 2, 1, kb, status, stream);
     g_launches.fetch_add(1);
     return ok ? BSP_OK : BSP_ERR_CUDA;
 }
@@ -647,6 +650,29 @@ int launch_gemm_fp8_packed(const void* A, const void* sfa, const void* B, const 
 }  // namespace bsp
 
 using namespace bsp;
+
+namespace {
+
+// Argument checks of one conversion; its input and output byte ranges go to `in_r` / `out_r`.
+int check_sf_job(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in, void* sf_out, int64_t ld_out,
+                 const char* in_r[2], const char* out_r[2]) {
+    if (!sf_in || !sf_out || mn <= 0 || kb <= 0 || (in_kind != 0 && in_kind != 1)) return BSP_ERR_ARG;
+    if (ld_in < kb || ld_out < mn) return BSP_ERR_SHAPE;
+    if ((ld_out * 2) % 16 || !aligned16(sf_out)) return BSP_ERR_ALIGN;
+    if (in_kind == 0 && (reinterpret_cast<uintptr_t>(sf_in) & 3u)) return BSP_ERR_ALIGN;
+    const int words = (kb + 1) / 2;
+    in_r[0] = static_cast<const char*>(sf_in);
+    in_r[1] = in_r[0] + ((int64_t)(mn - 1) * ld_in + kb) * (in_kind == 0 ? 4 : 1);
+    out_r[0] = static_cast<const char*>(sf_out);
+    out_r[1] = out_r[0] + (int64_t)words * ld_out * 2;
+    if (in_r[0] < out_r[1] && out_r[0] < in_r[1]) return BSP_ERR_ARG;  // overlapping buffers
+    if ((kb + kSfTileKB - 1) / kSfTileKB > 65535) return BSP_ERR_UNSUPPORTED;
+    return BSP_OK;
+}
+
+bool overlap(const char* const a[2], const char* const b[2]) { return a[0] < b[1] && b[0] < a[1]; }
+
+}  // namespace
 
 extern "C" {
 
@@ -804,21 +830,28 @@ int m_grouped_gemm_fp8_nt_masked(const void* A, const void* sfa, const void* B, 
 
 int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t ld_in, void* sf_out, int64_t ld_out,
                        void* stream) {
-    if (!sf_in || !sf_out || mn <= 0 || kb <= 0 || (in_kind != 0 && in_kind != 1)) return BSP_ERR_ARG;
-    if (ld_in < kb || ld_out < mn) return BSP_ERR_SHAPE;
-    if ((ld_out * 2) % 16 || !aligned16(sf_out)) return BSP_ERR_ALIGN;
-    if (in_kind == 0 && (reinterpret_cast<uintptr_t>(sf_in) & 3u)) return BSP_ERR_ALIGN;
-    const int words = (kb + 1) / 2;
-    const char* ib = static_cast<const char*>(sf_in);
-    const char* ie = ib + ((int64_t)(mn - 1) * ld_in + kb) * (in_kind == 0 ? 4 : 1);
-    const char* ob = static_cast<const char*>(sf_out);
-    const char* oe = ob + (int64_t)words * ld_out * 2;
-    if (ib < oe && ob < ie) return BSP_ERR_ARG;  // overlapping buffers
-    if ((kb + kSfTileKB - 1) / kSfTileKB > 65535) return BSP_ERR_UNSUPPORTED;
+    const char *in_r[2], *out_r[2];
+    BSP_TRY(check_sf_job(sf_in, in_kind, mn, kb, ld_in, sf_out, ld_out, in_r, out_r));
     DeviceCtx* ctx;
     BSP_TRY(ensure_ctx(&ctx));
     const bool ok = launch_sf_transform(sf_in, in_kind, mn, kb, ld_in, static_cast<uint16_t*>(sf_out), ld_out,
                                         ctx->status, static_cast<cudaStream_t>(stream));
+    g_launches.fetch_add(1);
+    return ok ? BSP_OK : BSP_ERR_CUDA;
+}
+
+int transform_sf_ue8m0_pair(const void* sf_a, int mn_a, int64_t ld_in_a, void* out_a, int64_t ld_out_a,
+                            const void* sf_b, int mn_b, int64_t ld_in_b, void* out_b, int64_t ld_out_b, int in_kind,
+                            int kb, void* stream) {
+    const char *in_a[2], *oa[2], *in_b[2], *ob[2];
+    BSP_TRY(check_sf_job(sf_a, in_kind, mn_a, kb, ld_in_a, out_a, ld_out_a, in_a, oa));
+    BSP_TRY(check_sf_job(sf_b, in_kind, mn_b, kb, ld_in_b, out_b, ld_out_b, in_b, ob));
+    if (overlap(oa, ob) || overlap(oa, in_b) || overlap(ob, in_a)) return BSP_ERR_ARG;
+    DeviceCtx* ctx;
+    BSP_TRY(ensure_ctx(&ctx));
+    const SfJob jobs[2] = {{sf_a, ld_in_a, static_cast<uint16_t*>(out_a), ld_out_a, mn_a},
+                           {sf_b, ld_in_b, static_cast<uint16_t*>(out_b), ld_out_b, mn_b}};
+    const bool ok = launch_sf_transform(jobs, 2, in_kind, kb, ctx->status, static_cast<cudaStream_t>(stream));
     g_launches.fetch_add(1);
     return ok ? BSP_OK : BSP_ERR_CUDA;
 }

@@ -14,9 +14,11 @@ namespace detail {
 int status_word(int** out);
 void note_launch();
 
-// SF words from uint8 UE8M0 bytes [mn][ld_in] into int16 [ceil(kb/2)][ld_out]; faults latch `status`.
-int launch_sf_transform_u8(const void* in, int mn, int kb, int64_t ld_in, void* out, int64_t ld_out, int* status,
-                           cudaStream_t stream);
+// SF words from two uint8 UE8M0 byte tensors [mn_x][ld_in_x] (the same kb) into int16
+// [ceil(kb/2)][ld_out_x], in one launch; faults latch `status`.
+int launch_sf_transform_u8_pair(const void* in_a, int mn_a, int64_t ld_in_a, void* out_a, int64_t ld_out_a,
+                                const void* in_b, int mn_b, int64_t ld_in_b, void* out_b, int64_t ld_out_b, int kb,
+                                int* status, cudaStream_t stream);
 
 // Bytes of scratch the FP8 GEMM lays its scale chunks out in, for this problem.
 int64_t gemm_fp8_scale_scratch_bytes(int M, int N, int K, int sfb_gran_n);

@@ -78,9 +78,8 @@ extern "C" int gemm_fp8_nt_noalloc(const void* A, const void* sfa_e8m0, const vo
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the status word must start at zero for this call; the scratch is fully rewritten below
     if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return BSP_ERR_CUDA;
-    if (const int rc = bsp::detail::launch_sf_transform_u8(sfa_e8m0, M, kb, ld_sfa_in, sfa_w, ld_a, status, st))
-        return rc;
-    if (const int rc = bsp::detail::launch_sf_transform_u8(sfb_e8m0, mn_b, kb, ld_sfb_in, sfb_w, ld_b, status, st))
+    if (const int rc = bsp::detail::launch_sf_transform_u8_pair(sfa_e8m0, M, ld_sfa_in, sfa_w, ld_a, sfb_e8m0, mn_b,
+                                                                ld_sfb_in, sfb_w, ld_b, kb, status, st))
         return rc;
     return bsp::detail::launch_gemm_fp8_packed(A, sfa_w, B, sfb_w, D, M, N, K, lda, ldb, ldd, ld_a, ld_b,
                                                sfb_gran_n, status, sfa_w + off_chunks,

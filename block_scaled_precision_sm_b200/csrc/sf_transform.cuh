@@ -49,13 +49,32 @@ struct SfVec<1> {
     static __device__ __forceinline__ uint32_t word(const T& v, int) { return v; }
 };
 
+// One tensor to convert: scales [mn][kb] at `in` (row stride ld_in) -> words at `out` (ld_out).
+struct SfJob {
+    const void* in;
+    int64_t ld_in;
+    uint16_t* out;
+    int64_t ld_out;
+    int mn;
+};
+// Up to two tensors with the same kb and input kind, converted by one launch (blockIdx.z
+// picks the tensor), so that independent conversions share one launch and one round trip.
+struct SfJobs {
+    SfJob job[2];
+};
+
 // IN_KIND 0: fp32 power-of-two scales (UE8M0 byte = biased fp32 exponent);
 // IN_KIND 1: uint8 UE8M0 bytes.  VEC: bytes per global load (16, 8 or 4 for fp32; 16, 8, 4 or
-// 1 for bytes); the row stride ld_in and the base are multiples of VEC bytes.
+// 1 for bytes); every job's row stride ld_in and base are multiples of VEC bytes.
 template <int IN_KIND, int VEC>
-__global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const void* __restrict__ in, int mn, int kb,
-                                                                  int64_t ld_in, uint16_t* __restrict__ out,
-                                                                  int64_t ld_out, int* status) {
+__global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const SfJobs jobs, int kb, int* status) {
+    const SfJob jb = blockIdx.z == 0 ? jobs.job[0] : jobs.job[1];
+    // the grid covers the larger job: row tiles past this job's end have nothing to do
+    if ((int64_t)blockIdx.x * kSfTileMN >= jb.ld_out) return;
+    const void* __restrict__ in = jb.in;
+    uint16_t* __restrict__ out = jb.out;
+    const int mn = jb.mn;
+    const int64_t ld_in = jb.ld_in, ld_out = jb.ld_out;
     constexpr int ES = IN_KIND == 0 ? 4 : 1;       // input element bytes
     constexpr int EV = VEC / ES;                   // elements per load
     static_assert(EV >= 1 && kSfTileKB % EV == 0, "vector width");
@@ -189,8 +208,7 @@ inline int sf_transform_vec(const void* in, int in_kind, int64_t ld_in) {
 }
 
 template <int IN_KIND, int VEC>
-inline bool launch_sf_transform_vec(dim3 grid, const void* in, int mn, int kb, int64_t ld_in, uint16_t* out,
-                                    int64_t ld_out, int* status, cudaStream_t stream) {
+inline bool launch_sf_transform_vec(dim3 grid, const SfJobs& jobs, int kb, int* status, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -200,28 +218,41 @@ inline bool launch_sf_transform_vec(dim3 grid, const void* in, int mn, int kb, i
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sf_transform_kernel<IN_KIND, VEC>, in, mn, kb, ld_in, out, ld_out, status) ==
-           cudaSuccess;
+    return cudaLaunchKernelEx(&cfg, sf_transform_kernel<IN_KIND, VEC>, jobs, kb, status) == cudaSuccess;
 }
 
-// Launch on `stream` (programmatic serialisation: the kernel waits for the one before it);
-// false if the launch failed or the grid is too large.
-inline bool launch_sf_transform(const void* in, int in_kind, int mn, int kb, int64_t ld_in, uint16_t* out,
-                                int64_t ld_out, int* status, cudaStream_t stream) {
-    const dim3 grid((unsigned)((ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB));
+// Launch `count` (1 or 2) jobs on `stream` (programmatic serialisation: the kernel waits for
+// the one before it); false if the launch failed or the grid is too large.
+inline bool launch_sf_transform(const SfJob* job, int count, int in_kind, int kb, int* status, cudaStream_t stream) {
+    SfJobs jobs = {};
+    int64_t ld_max = 0;
+    int vec = 16;
+    for (int i = 0; i < count; ++i) {
+        jobs.job[i] = job[i];
+        ld_max = job[i].ld_out > ld_max ? job[i].ld_out : ld_max;
+        const int v = sf_transform_vec(job[i].in, in_kind, job[i].ld_in);
+        vec = v < vec ? v : vec;
+    }
+    const dim3 grid((unsigned)((ld_max + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB),
+                    (unsigned)count);
     if (grid.y > 65535u) return false;
-    const int vec = sf_transform_vec(in, in_kind, ld_in);
     bool ok;
     if (in_kind == 0)
-        ok = vec == 16  ? launch_sf_transform_vec<0, 16>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
-             : vec == 8 ? launch_sf_transform_vec<0, 8>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
-                        : launch_sf_transform_vec<0, 4>(grid, in, mn, kb, ld_in, out, ld_out, status, stream);
+        ok = vec == 16  ? launch_sf_transform_vec<0, 16>(grid, jobs, kb, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<0, 8>(grid, jobs, kb, status, stream)
+                        : launch_sf_transform_vec<0, 4>(grid, jobs, kb, status, stream);
     else
-        ok = vec == 16  ? launch_sf_transform_vec<1, 16>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
-             : vec == 8 ? launch_sf_transform_vec<1, 8>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
-             : vec == 4 ? launch_sf_transform_vec<1, 4>(grid, in, mn, kb, ld_in, out, ld_out, status, stream)
-                        : launch_sf_transform_vec<1, 1>(grid, in, mn, kb, ld_in, out, ld_out, status, stream);
+        ok = vec == 16  ? launch_sf_transform_vec<1, 16>(grid, jobs, kb, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<1, 8>(grid, jobs, kb, status, stream)
+             : vec == 4 ? launch_sf_transform_vec<1, 4>(grid, jobs, kb, status, stream)
+                        : launch_sf_transform_vec<1, 1>(grid, jobs, kb, status, stream);
     return ok && cudaGetLastError() == cudaSuccess;
+}
+
+inline bool launch_sf_transform(const void* in, int in_kind, int mn, int kb, int64_t ld_in, uint16_t* out,
+                                int64_t ld_out, int* status, cudaStream_t stream) {
+    const SfJob job{in, ld_in, out, ld_out, mn};
+    return launch_sf_transform(&job, 1, in_kind, kb, status, stream);
 }
 
 }  // namespace bsp

@@ -94,6 +94,39 @@ def transform_sf_ue8m0(sf: torch.Tensor, ld_out: int | None = None, stream=None,
     return out
 
 
+def _sf_kind(sf: torch.Tensor) -> int:
+    if sf.dtype == torch.float32:
+        return 0
+    if sf.dtype == torch.uint8:
+        return 1
+    raise ValueError("scale factors must be float32 (powers of two) or uint8 (UE8M0 bytes)")
+
+
+def _sf_out(out, sf, mn, kb, name):
+    if out is None:
+        return torch.empty(((kb + 1) // 2, sf_ld(mn)), dtype=torch.int16, device=sf.device)
+    _rowmajor(out, name)
+    if out.dtype != torch.int16 or out.shape[0] != (kb + 1) // 2 or out.shape[1] < mn:
+        raise ValueError(f"{name} must be int16 [ceil(KB/2), >= MN]")
+    return out
+
+
+@_on_tensor_device
+def transform_sf_ue8m0_pair(sf_a: torch.Tensor, sf_b: torch.Tensor, out_a: torch.Tensor | None = None,
+                            out_b: torch.Tensor | None = None, stream=None):
+    """Two transform_sf_ue8m0 conversions with the same dtype and KB (a GEMM's A and B scales)
+    in one launch; returns (out_a, out_b)."""
+    kind = _sf_kind(sf_a)
+    if _sf_kind(sf_b) != kind or sf_a.dim() != 2 or sf_b.dim() != 2 or sf_a.shape[1] != sf_b.shape[1]:
+        raise ValueError("sf_a and sf_b must be [MN, KB] of one dtype with the same KB")
+    (mn_a, kb), mn_b = sf_a.shape, sf_b.shape[0]
+    ld_a, ld_b = _rowmajor(sf_a, "sf_a"), _rowmajor(sf_b, "sf_b")
+    out_a, out_b = _sf_out(out_a, sf_a, mn_a, kb, "out_a"), _sf_out(out_b, sf_b, mn_b, kb, "out_b")
+    _lib.call("transform_sf_ue8m0_pair", _ptr(sf_a), mn_a, ld_a, _ptr(out_a), out_a.stride(0), _ptr(sf_b), mn_b,
+              ld_b, _ptr(out_b), out_b.stride(0), kind, kb, _stream(stream))
+    return out_a, out_b
+
+
 def is_packed_sf(sf: torch.Tensor, mn: int, kb: int) -> bool:
     """True if `sf` already is the packed layout for MN scale rows and KB blocks."""
     return (sf.dtype == torch.int16 and sf.dim() == 2 and sf.shape[0] == (kb + 1) // 2
@@ -108,6 +141,16 @@ def packed_sf(sf: torch.Tensor, mn: int, kb: int, stream=None) -> torch.Tensor:
     if sf.dim() != 2 or tuple(sf.shape) != (mn, kb):
         raise ValueError(f"scale factors must be packed int16 [{(kb + 1) // 2}, >={mn}] or [{mn}, {kb}]")
     return transform_sf_ue8m0(sf, stream=stream)
+
+
+def _packed_pair(sfa, mn_a, sfb, mn_b, kb, stream):
+    """Both operands' scales packed: each reused if it already is, and converted together in
+    one launch when neither is."""
+    if (not is_packed_sf(sfa, mn_a, kb) and not is_packed_sf(sfb, mn_b, kb) and sfa.dtype == sfb.dtype
+            and sfa.dim() == 2 and tuple(sfa.shape) == (mn_a, kb) and sfb.dim() == 2
+            and tuple(sfb.shape) == (mn_b, kb)):
+        return transform_sf_ue8m0_pair(sfa, sfb, stream=stream)
+    return packed_sf(sfa, mn_a, kb, stream), packed_sf(sfb, mn_b, kb, stream)
 
 
 def _out(D, m, n, device):
@@ -137,8 +180,7 @@ def gemm_fp8_nt(A, sfa, B, sfb, D=None, sfb_gran_n: int = 128, stream=None) -> t
     lda, ldb = _rowmajor(A8, "A"), _rowmajor(B8, "B")
     (m, k), n = A8.shape, B8.shape[0]
     kb = k // 128
-    sfa = packed_sf(sfa, m, kb, stream)
-    sfb = packed_sf(sfb, -(-n // sfb_gran_n), kb, stream)
+    sfa, sfb = _packed_pair(sfa, m, sfb, -(-n // sfb_gran_n), kb, stream)
     D = _out(D, m, n, A8.device)
     _lib.call("gemm_fp8_nt", _ptr(A8), _ptr(sfa), _ptr(B8), _ptr(sfb), _ptr(D), m, n, k, lda, ldb,
               _rowmajor(D, "D"), sfa.stride(0), sfb.stride(0), sfb_gran_n, _stream(stream))
@@ -152,8 +194,7 @@ def gemm_fp4_nt(A, sfa, B, sfb, D=None, stream=None) -> torch.Tensor:
     lda, ldb = _rowmajor(A8, "A"), _rowmajor(B8, "B")
     m, k, n = A8.shape[0], A8.shape[1] * 2, B8.shape[0]
     kb = k // 32
-    sfa = packed_sf(sfa, m, kb, stream)
-    sfb = packed_sf(sfb, n, kb, stream)
+    sfa, sfb = _packed_pair(sfa, m, sfb, n, kb, stream)
     D = _out(D, m, n, A8.device)
     _lib.call("gemm_fp4_nt", _ptr(A8), _ptr(sfa), _ptr(B8), _ptr(sfb), _ptr(D), m, n, k, lda, ldb,
               _rowmajor(D, "D"), sfa.stride(0), sfb.stride(0), _stream(stream))

@@ -164,6 +164,17 @@ int transform_sf_ue8m0(const void* sf_in, int in_kind, int mn, int kb, int64_t l
                        void* sf_out, int64_t ld_out, void* stream);
 
 /*
+ * transform_sf_ue8m0_pair — two independent conversions of transform_sf_ue8m0 with the same
+ * in_kind and kb (a GEMM's A and B scales) in one launch: sf_a [mn_a][kb] (row stride
+ * ld_in_a) into out_a int16 [ceil(kb/2)][ld_out_a], and likewise for b.  Each tensor follows
+ * the rules of transform_sf_ue8m0; no output may overlap the other output or either input.
+ * The results are the bytes the two single calls give.
+ */
+int transform_sf_ue8m0_pair(const void* sf_a, int mn_a, int64_t ld_in_a, void* out_a, int64_t ld_out_a,
+                            const void* sf_b, int mn_b, int64_t ld_in_b, void* out_b, int64_t ld_out_b,
+                            int in_kind, int kb, void* stream);
+
+/*
  * quantize_fp8_ue8m0 — the step before the GEMM: real values to E4M3 codes with one
  * power-of-two UE8M0 scale per block, the scales written straight into the SF-word layout
  * ("DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Fatores de escala FP8

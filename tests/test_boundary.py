@@ -77,6 +77,13 @@ def test_rejects_bad_arguments_without_gpu(lib):
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 4, None) == -3
     assert lib.transform_sf_ue8m0(good, 1, 8, 8, 8, vp(0x20000), 12, None) == -2
     assert lib.transform_sf_ue8m0(good, 1, 64, 8, 8, vp(0x10010), 64, None) == -1
+    # the pair: kind, ld_out, alignment, and each output against the other output and inputs
+    pair = lib.transform_sf_ue8m0_pair
+    assert pair(good, 8, 8, vp(0x20000), 8, good, 8, 8, vp(0x30000), 8, 2, 8, None) == -1
+    assert pair(good, 8, 8, vp(0x20000), 8, good, 16, 8, vp(0x30000), 8, 1, 8, None) == -3
+    assert pair(good, 8, 8, vp(0x20000), 8, good, 8, 8, vp(0x30008), 8, 1, 8, None) == -2
+    assert pair(good, 8, 8, vp(0x20000), 8, good, 8, 8, vp(0x20010), 8, 1, 8, None) == -1
+    assert pair(vp(0x40000), 64, 8, vp(0x20000), 64, good, 8, 8, vp(0x40010), 8, 1, 8, None) == -1
     # masked grouped: max_m not a multiple of 128, G out of range, misaligned counts
     mm = vp(0x40000)
     assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, mm, 2, 100, 128, 128, 256, 8, 128,

@@ -77,6 +77,42 @@ def test_transform_vector_widths(ops, orc, kind, mn, kb, ld_in):
     assert np.array_equal(got.cpu().numpy(), orc.sf_pack(e, ld_out=ld_out))
 
 
+# Two conversions in one launch (a GEMM's A and B scales): the same bytes as two single calls
+# and as the oracle's packing, whichever tensor is larger, with different load widths and padded
+# outputs.
+@pytest.mark.parametrize("kind,mn_a,mn_b,kb,ld_in_a,ld_in_b", [("u8", 4096, 56, 128, 128, 128),
+                                                               ("u8", 37, 300, 5, 5, 8),
+                                                               ("fp32", 4096, 7168, 512, 512, 512),
+                                                               ("fp32", 129, 7, 3, 3, 4), ("u8", 1, 1, 1, 1, 1)])
+def test_transform_pair_matches_single_calls_and_oracle(ops, orc, kind, mn_a, mn_b, kb, ld_in_a, ld_in_b):
+    rng = np.random.default_rng(mn_a + 3 * mn_b + kb)
+    srcs, es = [], []
+    for mn, ld_in in ((mn_a, ld_in_a), (mn_b, ld_in_b)):
+        e = rng.integers(1, 255, size=(mn, kb), dtype=np.uint8)
+        full = np.zeros((mn, ld_in), np.uint8 if kind == "u8" else np.float32)
+        full[:, :kb] = e if kind == "u8" else np.ldexp(np.float32(1.0), e.astype(np.int32) - 127)
+        srcs.append(to_dev(full)[:, :kb])
+        es.append(e)
+    lds = [(mn_a + 7) // 8 * 8 + 8, (mn_b + 7) // 8 * 8 + 16]
+    outs = [torch.full(((kb + 1) // 2, ld), -1, dtype=torch.int16, device="cuda") for ld in lds]
+    ops.transform_sf_ue8m0_pair(srcs[0], srcs[1], out_a=outs[0], out_b=outs[1])
+    _status_ok(ops)
+    for src, e, out, ld in zip(srcs, es, outs, lds):
+        assert np.array_equal(out.cpu().numpy(), orc.sf_pack(e, ld_out=ld))
+        assert torch.equal(out, ops.transform_sf_ue8m0(src, ld_out=ld))
+
+
+def test_transform_pair_flags_nan_byte_in_either(ops, orc):
+    a = np.full((300, 6), 127, np.uint8)
+    b = np.full((20, 6), 127, np.uint8)
+    b[19, 0] = 0xFF
+    out_a, out_b = ops.transform_sf_ue8m0_pair(to_dev(a), to_dev(b))
+    assert ops.device_status() == -7
+    _status_ok(ops)  # cleared
+    assert np.array_equal(out_b.cpu().numpy(), orc.sf_pack(b, ld_out=out_b.shape[1]))
+    assert np.array_equal(out_a.cpu().numpy(), orc.sf_pack(a, ld_out=out_a.shape[1]))
+
+
 def test_transform_flags_bad_scale(ops):
     s = np.ones((16, 4), np.float32)
     s[3, 2] = 3.0
