@@ -55,7 +55,7 @@ _CSRC = "block_scaled_precision_sm_b200/csrc/"
 # the sources each profiled kernel depends on (device code and the host code that launches it)
 KERNEL_SOURCES = {
     "gemm": [_CSRC + f for f in ("gemm.cuh", "ptx.cuh", "sf_layout.cuh", "api.cu")],
-    "sf_transform": [_CSRC + f for f in ("sf_transform.cuh", "ptx.cuh", "api.cu")],
+    "sf_transform": [_CSRC + f for f in ("sf_transform.cuh", "ptx.cuh", "api.cu", "sf_batch.cu")],
     "quantize": [_CSRC + f for f in ("quantize.cuh", "quantize.cu")],
 }
 

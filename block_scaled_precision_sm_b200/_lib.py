@@ -19,6 +19,7 @@ SIGNATURES = {
     "m_grouped_gemm_fp8_nt_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i64, _i64, _i, _vp]),
     "transform_sf_ue8m0": (_i, [_vp, _i, _i, _i, _i64, _vp, _i64, _vp]),
     "transform_sf_ue8m0_pair": (_i, [_vp, _i, _i64, _vp, _i64, _vp, _i, _i64, _vp, _i64, _i, _i, _vp]),
+    "transform_sf_ue8m0_batched": (_i, [_vp, _i, _i, _i, _i, _i64, _i64, _vp, _i64, _i64, _vp]),
     "gemm_fp8_nt_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i64, _i64, _i64, _i64, _i64, _i, _vp]),
     "bsp_get_device_status": (_i, [_vp]),
     "bsp_status_string": (ctypes.c_char_p, [_i]),

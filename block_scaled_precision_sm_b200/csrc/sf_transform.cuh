@@ -57,10 +57,14 @@ struct SfJob {
     int64_t ld_out;
     int mn;
 };
-// Up to two tensors with the same kb and input kind, converted by one launch (blockIdx.z
-// picks the tensor), so that independent conversions share one launch and one round trip.
+// Tensors with the same kb and input kind converted by one launch, so that independent
+// conversions share one launch and one round trip; blockIdx.z picks the tensor.  Either a
+// table of up to two (in_zstride == 0), or a batch: tensor z is job[0] moved by z * in_zstride
+// input bytes and z * out_zstride output words.
 struct SfJobs {
     SfJob job[2];
+    int64_t in_zstride;
+    int64_t out_zstride;
 };
 
 // IN_KIND 0: fp32 power-of-two scales (UE8M0 byte = biased fp32 exponent);
@@ -68,7 +72,12 @@ struct SfJobs {
 // 1 for bytes); every job's row stride ld_in and base are multiples of VEC bytes.
 template <int IN_KIND, int VEC>
 __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const SfJobs jobs, int kb, int* status) {
-    const SfJob jb = blockIdx.z == 0 ? jobs.job[0] : jobs.job[1];
+    SfJob jb = blockIdx.z == 0 ? jobs.job[0] : jobs.job[1];
+    if (jobs.in_zstride != 0) {
+        jb = jobs.job[0];
+        jb.in = static_cast<const char*>(jb.in) + (int64_t)blockIdx.z * jobs.in_zstride;
+        jb.out += (int64_t)blockIdx.z * jobs.out_zstride;
+    }
     // the grid covers the larger job: row tiles past this job's end have nothing to do
     if ((int64_t)blockIdx.x * kSfTileMN >= jb.ld_out) return;
     const void* __restrict__ in = jb.in;
@@ -198,10 +207,11 @@ __global__ void __launch_bounds__(kSfThreads) sf_transform_kernel(const SfJobs j
     if (__any_sync(0xffffffffu, bad) && (t % 32) == 0) atomicCAS(status, 0, -7);
 }
 
-// Widest load (bytes) that the input's base address and row stride allow.
-inline int sf_transform_vec(const void* in, int in_kind, int64_t ld_in) {
+// Widest load (bytes) that the input's base address and row stride (and the stride between
+// the tensors of a batch) allow.
+inline int sf_transform_vec(const void* in, int in_kind, int64_t ld_in, int64_t zstride_bytes = 0) {
     const int es = in_kind == 0 ? 4 : 1;
-    const uint64_t a = reinterpret_cast<uintptr_t>(in) | (uint64_t)(ld_in * es);
+    const uint64_t a = reinterpret_cast<uintptr_t>(in) | (uint64_t)(ld_in * es) | (uint64_t)zstride_bytes;
     for (int v : {16, 8, 4})
         if (a % (uint64_t)v == 0) return v;
     return es == 4 ? 4 : 1;
@@ -221,6 +231,22 @@ inline bool launch_sf_transform_vec(dim3 grid, const SfJobs& jobs, int kb, int* 
     return cudaLaunchKernelEx(&cfg, sf_transform_kernel<IN_KIND, VEC>, jobs, kb, status) == cudaSuccess;
 }
 
+inline bool launch_sf_jobs(const SfJobs& jobs, dim3 grid, int vec, int in_kind, int kb, int* status,
+                           cudaStream_t stream) {
+    if (grid.y > 65535u || grid.z > 65535u) return false;
+    bool ok;
+    if (in_kind == 0)
+        ok = vec == 16  ? launch_sf_transform_vec<0, 16>(grid, jobs, kb, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<0, 8>(grid, jobs, kb, status, stream)
+                        : launch_sf_transform_vec<0, 4>(grid, jobs, kb, status, stream);
+    else
+        ok = vec == 16  ? launch_sf_transform_vec<1, 16>(grid, jobs, kb, status, stream)
+             : vec == 8 ? launch_sf_transform_vec<1, 8>(grid, jobs, kb, status, stream)
+             : vec == 4 ? launch_sf_transform_vec<1, 4>(grid, jobs, kb, status, stream)
+                        : launch_sf_transform_vec<1, 1>(grid, jobs, kb, status, stream);
+    return ok && cudaGetLastError() == cudaSuccess;
+}
+
 // Launch `count` (1 or 2) jobs on `stream` (programmatic serialisation: the kernel waits for
 // the one before it); false if the launch failed or the grid is too large.
 inline bool launch_sf_transform(const SfJob* job, int count, int in_kind, int kb, int* status, cudaStream_t stream) {
@@ -235,18 +261,21 @@ inline bool launch_sf_transform(const SfJob* job, int count, int in_kind, int kb
     }
     const dim3 grid((unsigned)((ld_max + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB),
                     (unsigned)count);
-    if (grid.y > 65535u) return false;
-    bool ok;
-    if (in_kind == 0)
-        ok = vec == 16  ? launch_sf_transform_vec<0, 16>(grid, jobs, kb, status, stream)
-             : vec == 8 ? launch_sf_transform_vec<0, 8>(grid, jobs, kb, status, stream)
-                        : launch_sf_transform_vec<0, 4>(grid, jobs, kb, status, stream);
-    else
-        ok = vec == 16  ? launch_sf_transform_vec<1, 16>(grid, jobs, kb, status, stream)
-             : vec == 8 ? launch_sf_transform_vec<1, 8>(grid, jobs, kb, status, stream)
-             : vec == 4 ? launch_sf_transform_vec<1, 4>(grid, jobs, kb, status, stream)
-                        : launch_sf_transform_vec<1, 1>(grid, jobs, kb, status, stream);
-    return ok && cudaGetLastError() == cudaSuccess;
+    return launch_sf_jobs(jobs, grid, vec, in_kind, kb, status, stream);
+}
+
+// `batch` tensors of the same shape, tensor z at job.in + z * in_zstride_bytes and job.out +
+// z * out_zstride words, in one launch (batch <= 65535).
+inline bool launch_sf_transform_batched(const SfJob& job, int batch, int64_t in_zstride_bytes, int64_t out_zstride,
+                                        int in_kind, int kb, int* status, cudaStream_t stream) {
+    SfJobs jobs = {};
+    jobs.job[0] = job;
+    jobs.in_zstride = batch > 1 ? in_zstride_bytes : 0;
+    jobs.out_zstride = batch > 1 ? out_zstride : 0;
+    const int vec = sf_transform_vec(job.in, in_kind, job.ld_in, jobs.in_zstride);
+    const dim3 grid((unsigned)((job.ld_out + kSfTileMN - 1) / kSfTileMN), (unsigned)((kb + kSfTileKB - 1) / kSfTileKB),
+                    (unsigned)batch);
+    return launch_sf_jobs(jobs, grid, vec, in_kind, kb, status, stream);
 }
 
 inline bool launch_sf_transform(const void* in, int in_kind, int mn, int kb, int64_t ld_in, uint16_t* out,

@@ -127,6 +127,24 @@ def transform_sf_ue8m0_pair(sf_a: torch.Tensor, sf_b: torch.Tensor, out_a: torch
     return out_a, out_b
 
 
+@_on_tensor_device
+def transform_sf_ue8m0_batched(sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """transform_sf_ue8m0 of every tensor of a stack [G, MN, KB] (fp32 or uint8) in one launch:
+    int16 words [G, ceil(KB/2), ld]."""
+    kind = _sf_kind(sf)
+    if sf.dim() != 3 or sf.stride(2) != 1 or sf.stride(1) < sf.shape[2]:
+        raise ValueError("sf must be [G, MN, KB] with KB contiguous")
+    g, mn, kb = sf.shape
+    if out is None:
+        out = torch.empty((g, (kb + 1) // 2, sf_ld(mn)), dtype=torch.int16, device=sf.device)
+    if (out.dtype != torch.int16 or out.dim() != 3 or out.shape[0] != g or out.shape[1] != (kb + 1) // 2
+            or out.shape[2] < mn or out.stride(2) != 1 or out.stride(1) < out.shape[2]):
+        raise ValueError("out must be int16 [G, ceil(KB/2), >= MN] with the last dimension contiguous")
+    _lib.call("transform_sf_ue8m0_batched", _ptr(sf), kind, g, mn, kb, sf.stride(1), sf.stride(0), _ptr(out),
+              out.stride(1), out.stride(0), _stream(stream))
+    return out
+
+
 def is_packed_sf(sf: torch.Tensor, mn: int, kb: int) -> bool:
     """True if `sf` already is the packed layout for MN scale rows and KB blocks."""
     return (sf.dtype == torch.int16 and sf.dim() == 2 and sf.shape[0] == (kb + 1) // 2
@@ -221,7 +239,7 @@ def m_grouped_gemm_fp8_nt_contiguous(A, sfa, B, sfb, m_indices, D=None, sfb_gran
     else:
         if sfb.dim() != 3 or tuple(sfb.shape) != (g, mn_b, kb):
             raise ValueError(f"sfb must be packed int16 [G, words, ld] or [{g}, {mn_b}, {kb}]")
-        sfb = torch.stack([transform_sf_ue8m0(sfb[i], stream=stream) for i in range(g)])
+        sfb = transform_sf_ue8m0_batched(sfb, stream=stream)
     D = _out(D, m, n, A8.device)
     if not D.is_contiguous():
         raise ValueError("D must be contiguous")
@@ -254,7 +272,7 @@ def m_grouped_gemm_fp8_nt_masked(A, sfa, B, sfb, masked_m, D=None, sfb_gran_n: i
     else:
         if sfb.dim() != 3 or tuple(sfb.shape) != (g, mn_b, kb):
             raise ValueError(f"sfb must be packed int16 [G, words, ld] or [{g}, {mn_b}, {kb}]")
-        sfb = torch.stack([transform_sf_ue8m0(sfb[i], stream=stream) for i in range(g)])
+        sfb = transform_sf_ue8m0_batched(sfb, stream=stream)
     if D is None:
         D = torch.empty((g, max_m, n), dtype=torch.bfloat16, device=A8.device)
     if D.dtype != torch.bfloat16 or tuple(D.shape) != (g, max_m, n) or not D.is_contiguous():

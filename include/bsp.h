@@ -175,6 +175,20 @@ int transform_sf_ue8m0_pair(const void* sf_a, int mn_a, int64_t ld_in_a, void* o
                             int in_kind, int kb, void* stream);
 
 /*
+ * transform_sf_ue8m0_batched — transform_sf_ue8m0 of `batch` same-shaped tensors (for example
+ * the per-expert B scales [G][mn][kb] of a grouped GEMM) in one launch: tensor z is read at
+ * sf_in + z * batch_stride_in (elements of the input kind) and written at
+ * sf_out + z * batch_stride_out (int16 words), each with the rules of transform_sf_ue8m0.
+ *   1 <= batch <= 65535.  For batch > 1: batch_stride_in >= (mn-1)*ld_in + kb,
+ *   batch_stride_out >= ceil(kb/2)*ld_out and batch_stride_out*2 a multiple of 16 bytes (the
+ *   strides are ignored when batch == 1).  The whole input and output ranges must not overlap.
+ * The results are the bytes `batch` single calls give.
+ */
+int transform_sf_ue8m0_batched(const void* sf_in, int in_kind, int batch, int mn, int kb, int64_t ld_in,
+                               int64_t batch_stride_in, void* sf_out, int64_t ld_out, int64_t batch_stride_out,
+                               void* stream);
+
+/*
  * quantize_fp8_ue8m0 — the step before the GEMM: real values to E4M3 codes with one
  * power-of-two UE8M0 scale per block, the scales written straight into the SF-word layout
  * ("DeepGEMM-Ascend cobre quantas operações no Ascend 950?", section "Fatores de escala FP8

@@ -84,6 +84,14 @@ def test_rejects_bad_arguments_without_gpu(lib):
     assert pair(good, 8, 8, vp(0x20000), 8, good, 8, 8, vp(0x30008), 8, 1, 8, None) == -2
     assert pair(good, 8, 8, vp(0x20000), 8, good, 8, 8, vp(0x20010), 8, 1, 8, None) == -1
     assert pair(vp(0x40000), 64, 8, vp(0x20000), 64, good, 8, 8, vp(0x40010), 8, 1, 8, None) == -1
+    # the batch: count, strides too small for a tensor, misaligned output stride, overlap, size
+    bat = lib.transform_sf_ue8m0_batched
+    assert bat(good, 1, 0, 8, 8, 8, 64, vp(0x200000), 8, 32, None) == -1
+    assert bat(good, 1, 4, 8, 8, 8, 63, vp(0x200000), 8, 32, None) == -3
+    assert bat(good, 1, 4, 8, 8, 8, 64, vp(0x200000), 8, 31, None) == -3
+    assert bat(good, 1, 4, 8, 8, 8, 64, vp(0x200000), 8, 36, None) == -2
+    assert bat(good, 1, 4, 8, 8, 8, 64, vp(0x10080), 8, 32, None) == -1
+    assert bat(good, 1, 70000, 8, 8, 8, 64, vp(0x20000000), 8, 32, None) == -4
     # masked grouped: max_m not a multiple of 128, G out of range, misaligned counts
     mm = vp(0x40000)
     assert lib.m_grouped_gemm_fp8_nt_masked(good, good, good, good, good, mm, 2, 100, 128, 128, 256, 8, 128,

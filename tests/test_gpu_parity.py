@@ -113,6 +113,47 @@ def test_transform_pair_flags_nan_byte_in_either(ops, orc):
     assert np.array_equal(out_a.cpu().numpy(), orc.sf_pack(a, ld_out=out_a.shape[1]))
 
 
+# A stack of same-shaped tensors in one launch (per-expert B scales): each tensor the bytes a
+# single call and the oracle give, with gaps between the input rows and between the tensors on
+# both sides, and a batch of one.
+@pytest.mark.parametrize("kind,g,mn,kb,row_pad,gap_in,ld_pad,gap_out", [("u8", 32, 32, 56, 0, 0, 0, 0),
+                                                                        ("u8", 5, 300, 7, 1, 13, 8, 16),
+                                                                        ("fp32", 3, 129, 5, 3, 4, 0, 8),
+                                                                        ("fp32", 1, 40, 512, 0, 0, 16, 0)])
+def test_transform_batched_matches_single_calls_and_oracle(ops, orc, kind, g, mn, kb, row_pad, gap_in, ld_pad,
+                                                           gap_out):
+    rng = np.random.default_rng(g * mn + kb)
+    e = rng.integers(1, 255, size=(g, mn, kb), dtype=np.uint8)
+    ld_in = kb + row_pad
+    flat = np.zeros(g * (mn * ld_in + gap_in), np.uint8 if kind == "u8" else np.float32)
+    full = np.lib.stride_tricks.as_strided(flat, shape=(g, mn, ld_in),
+                                           strides=(flat.itemsize * (mn * ld_in + gap_in), flat.itemsize * ld_in,
+                                                    flat.itemsize))
+    full[:, :, :kb] = e if kind == "u8" else np.ldexp(np.float32(1.0), e.astype(np.int32) - 127)
+    dflat = to_dev(flat)
+    src = dflat.as_strided((g, mn, kb), (mn * ld_in + gap_in, ld_in, 1))
+    words, ld = (kb + 1) // 2, (mn + 7) // 8 * 8 + ld_pad
+    oflat = torch.full((g * (words * ld + gap_out),), -1, dtype=torch.int16, device="cuda")
+    out = oflat.as_strided((g, words, ld), (words * ld + gap_out, ld, 1))
+    ops.transform_sf_ue8m0_batched(src, out=out)
+    _status_ok(ops)
+    got = out.cpu().numpy()
+    for z in range(g):
+        assert np.array_equal(got[z], orc.sf_pack(e[z], ld_out=ld)), z
+        assert torch.equal(out[z], ops.transform_sf_ue8m0(src[z], ld_out=ld)), z
+    if gap_out:  # the gaps between output tensors are not written
+        gaps = oflat.view(g, -1)[:, words * ld:].cpu().numpy()
+        assert (gaps == -1).all()
+
+
+def test_transform_batched_flags_nan_byte(ops):
+    e = np.full((4, 20, 6), 127, np.uint8)
+    e[2, 19, 5] = 0xFF
+    ops.transform_sf_ue8m0_batched(to_dev(e))
+    assert ops.device_status() == -7
+    _status_ok(ops)  # cleared
+
+
 def test_transform_flags_bad_scale(ops):
     s = np.ones((16, 4), np.float32)
     s[3, 2] = 3.0
