@@ -215,7 +215,7 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
     a.ws = ws;
     a.tail_count = count;
     a.tail_claim = count ? count + tail_counters<C>(p) : nullptr;
-    a.group_m = 16;
+    a.group_m = 8;  // raster groups of 8 row blocks: measured ~1 % faster than 16 or 4 at 4096x7168x16384
     a.status = ctx.status;
     a.timeout_ns = g_timeout_ns.load();
     const int workers = a.num_work < max_workers ? a.num_work : max_workers;
